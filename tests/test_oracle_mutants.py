@@ -1,0 +1,171 @@
+"""The pins are strong enough: each plausible mistake planted in a copy of an
+oracle function (dropped term, wrong sign, transposed operand, wrong index,
+wrong rounding, wrong group axis, wrong nibble order) fails at least one pin.
+
+The mutants live here, on the CPU, and are never used by anything else.
+"""
+import numpy as np
+import pytest
+
+import oracle as orc
+from tests import oracle_checks as ck
+
+
+# ---------------- recurrence mutants ----------------
+
+def _step_factory(kind):
+    def step(S, q, k, v, alpha, beta):
+        S = np.asarray(S, dtype=np.float64)
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        a = np.asarray(alpha, dtype=np.float64)[:, None, None]
+        b = np.asarray(beta, dtype=np.float64)[:, None, None]
+        d_k = S.shape[-1]
+        kk = k[:, :, None] * k[:, None, :]
+        sign = 1.0 if kind == "sign" else -1.0
+        trans = np.eye(d_k)[None] + sign * b * kk
+        decay = 1.0 if kind == "no_alpha" else a
+        prod = np.matmul(S, trans) if kind != "left_multiply" else np.matmul(trans[:, :S.shape[1], :S.shape[1]], S)
+        write = v[:, :, None] * k[:, None, :]
+        if kind == "alpha_on_write":
+            write = a * write
+        if kind == "beta_dropped_write":
+            S_new = decay * prod + write
+        else:
+            S_new = decay * prod + b * write
+        o = np.matmul(S_new, q[:, :, None])[:, :, 0]
+        if kind == "o_before_update":
+            o = np.matmul(S, q[:, :, None])[:, :, 0]
+        return S_new, o
+    return step
+
+
+STEP_MUTANTS = ["sign", "no_alpha", "left_multiply", "alpha_on_write", "beta_dropped_write",
+                "o_before_update"]
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except (AssertionError, ValueError, IndexError):
+        return True
+    return False
+
+
+@pytest.mark.parametrize("kind", STEP_MUTANTS)
+def test_step_mutant_is_caught(kind):
+    mutant = _step_factory(kind)
+    caught = (_fails(ck.check_gdn_golden, mutant) or _fails(ck.check_gdn_bruteforce, mutant)
+              or _fails(ck.check_gdn_closed_forms, mutant))
+    assert caught, kind
+
+
+def _chunk_factory(kind):
+    def chunk(S0, K, V, alpha, beta, q=None):
+        N, n, _ = K.shape
+        al, be = np.asarray(alpha, float), np.asarray(beta, float)
+        gam = np.ones((N, n + 1, n + 1))
+        for t in range(1, n + 1):
+            for s in range(0, t):
+                lo = s + 1 if kind == "gamma_index" else s
+                gam[:, t, s] = np.prod(al[:, lo:t], axis=1)
+        gamma = gam[:, 1:, 0]
+        X = np.matmul(S0, np.swapaxes(K, 1, 2))
+        gram = np.matmul(K, np.swapaxes(K, 1, 2))
+        rhs = be[:, :, None] * (V - gamma[:, :, None] * np.swapaxes(X, 1, 2))
+        U = np.zeros_like(rhs)
+        for t in range(n):
+            acc = rhs[:, t, :].copy()
+            for s in range(t):
+                a_ts = be[:, t] * gam[:, t + 1, s + 1] * gram[:, t, s]
+                if kind == "sign":
+                    acc += a_ts[:, None] * U[:, s, :]
+                elif kind == "beta_of_s":
+                    acc -= (be[:, s] * gam[:, t + 1, s + 1] * gram[:, t, s])[:, None] * U[:, s, :]
+                else:
+                    acc -= a_ts[:, None] * U[:, s, :]
+            U[:, t, :] = acc
+        g_last = gam[:, n, 1:]
+        if kind == "no_final_decay":
+            g_last = np.ones_like(g_last)
+        S_n = gam[:, n, 0][:, None, None] * S0 + np.matmul(np.swapaxes(g_last[:, :, None] * U, 1, 2), K)
+        kq = np.matmul(K, q[:, :, None])[:, :, 0]
+        o = gam[:, n, 0][:, None] * np.matmul(S0, q[:, :, None])[:, :, 0] + np.sum((g_last * kq)[:, :, None] * U, axis=1)
+        return S_n, U, o
+    return chunk
+
+
+@pytest.mark.parametrize("kind", ["sign", "gamma_index", "beta_of_s", "no_final_decay"])
+def test_chunk_mutant_is_caught(kind):
+    assert _fails(ck.check_chunk_vs_sequential, _chunk_factory(kind), orc.gdn_step), kind
+
+
+# ---------------- encoder mutants ----------------
+
+def _quant_factory(kind):
+    def quantize(S, bits, axis="col"):
+        S = np.asarray(S, dtype=np.float32)
+        qmax = {4: 7, 8: 127}[bits]
+        red = -2 if axis == "col" else -1
+        if kind == "axis_swapped":
+            red = -1 if axis == "col" else -2
+        finite = np.isfinite(S).all(axis=red, keepdims=True)
+        absS = np.where(np.isfinite(S), np.abs(S), np.float32(0))
+        amax = absS.max(axis=red, keepdims=True).astype(np.float32)
+        div = np.float32(qmax + 1 if kind == "qmax_plus_one" else qmax)
+        s32 = (amax / div).astype(np.float32)
+        with np.errstate(over="ignore"):
+            s16 = s32.astype(np.float16)
+        s16 = np.where((amax > 0) & (s16 == 0), np.float16(2 ** -24), s16)
+        s16 = np.where(np.isinf(s16), np.float16(65504), s16)
+        sf = s16.astype(np.float32) if kind != "unrounded_scale" else s32
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = (S / np.where(sf == 0, np.float32(1), sf)).astype(np.float32)
+        if kind == "half_up":
+            codes = np.floor(ratio + np.float32(0.5))
+        elif kind == "truncate":
+            codes = np.trunc(ratio)
+        else:
+            codes = np.rint(ratio)
+        lo = -qmax - 1 if kind == "asymmetric_clamp" else -qmax
+        codes = np.clip(codes, lo, qmax)
+        codes = np.where(sf == 0, 0, codes)
+        codes = np.where(finite, codes, 0).astype(np.int8)
+        s16 = np.where(finite, s16, np.float16(np.nan)).astype(np.float16)
+        flags = 0 if finite.all() else orc.FLAG_NONFINITE
+        return codes, np.squeeze(s16, axis=red), flags
+    return quantize
+
+
+@pytest.mark.parametrize("kind", ["axis_swapped", "qmax_plus_one", "unrounded_scale", "half_up",
+                                  "truncate", "asymmetric_clamp"])
+def test_encoder_mutant_is_caught(kind):
+    q = _quant_factory(kind)
+    caught = (_fails(ck.check_encoder_golden, q, orc.pack_codes)
+              or _fails(ck.check_encoder_bruteforce, q)
+              or _fails(ck.check_encoder_invariants, q, orc.dequantize)
+              or _fails(ck.check_encoder_special_cases, q, orc.FLAG_NONFINITE, orc.FLAG_SCALE_OVERFLOW))
+    assert caught, kind
+
+
+def test_unmutated_copy_passes():
+    """The mutant factory without a mutation is the oracle: every pin passes,
+    so the failures above come from the planted mistakes alone."""
+    q = _quant_factory("none")
+    ck.check_encoder_golden(q, orc.pack_codes)
+    ck.check_encoder_bruteforce(q)
+    ck.check_encoder_invariants(q, orc.dequantize)
+    ck.check_chunk_vs_sequential(_chunk_factory("none"), orc.gdn_step)
+    ck.check_gdn_golden(_step_factory("none"))
+    ck.check_gdn_bruteforce(_step_factory("none"))
+    ck.check_gdn_closed_forms(_step_factory("none"))
+
+
+def test_pack_mutant_is_caught():
+    def pack_swapped(codes, bits):
+        codes = np.asarray(codes, dtype=np.int8)
+        if bits == 8:
+            return codes.view(np.uint8).copy()
+        lo = codes[..., 1::2].astype(np.int16) & 0xF
+        hi = codes[..., 0::2].astype(np.int16) & 0xF
+        return (lo | (hi << 4)).astype(np.uint8)
+    assert _fails(ck.check_encoder_golden, orc.quantize, pack_swapped)
