@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Throughput of PACE periodic low-bit recurrent-state decode on one node.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl pace|reference]
+
+One *step* is one period of the hot path over the whole pool: P decode
+launches (one token for each of the B x H heads) followed by one commit
+launch.  The default workload is the concurrency-stress configuration
+(B=4096 sequences, H=48 heads, d_k=d_v=128, P=8, 25% INT8 heads, bf16 io),
+whose 2.06 GB state pool is far larger than the 126 MB L2, so no L2 flush is
+needed between steps.  The state is first warmed by a 512-token unquantised
+fp32 prefill (pace_gdn_step_f32), then encoded into the pool.
+
+Printed: one JSON line (rank 0).  ``value`` is head-tokens/s over all ranks
+(each rank holds its own full pool: weak scaling; no collective on the data
+path).  Kernel durations come from CUDA events on the launching stream.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HBM_FALLBACK_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128, help="timed periods (128 x P=8 = 1024 tokens)")
+    ap.add_argument("--warmup", type=int, default=3, help="untimed periods before timing")
+    ap.add_argument("--impl", choices=["pace", "reference"], default="pace")
+    ap.add_argument("--workload", default="concurrency_stress")
+    ap.add_argument("--period", type=int, default=None, help="override P")
+    ap.add_argument("--prefill", type=int, default=None, help="warm-up prefill tokens (default: workload's)")
+    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-compare", action="store_true", help="skip the bf16-state comparison path")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-slots", type=int, default=32)
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, "fallback"
+
+
+def kernel_source_digest():
+    csrc = os.path.join(ROOT, "bit_recurrent_state_pace_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, digest: str):
+    """DRAM bytes per launch recorded by an ncu capture of the same kernel
+    sources (profiles/*.txt lines 'traffic <kernel> <bytes> <digest>')."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith(".txt"):
+            continue
+        with open(os.path.join(pdir, fn)) as f:
+            for line in f:
+                tok = line.split()
+                if len(tok) == 4 and tok[0] == "traffic" and tok[1] == kernel and tok[3] == digest:
+                    return float(tok[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while timing."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx.append(float(p[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, p[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample_rate(w, bits, slots: int, seed: int):
+    """The fp64 oracle as it stands, on `slots` whole sequences (all H heads)
+    for one period of P tokens plus the commit; head-tokens per second."""
+    import numpy as np
+    import torch
+    import oracle as orc
+    import pace_synth
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    sub = w.replace(B=slots)
+    heads = [(b, h) for b in range(slots) for h in range(w.H)]
+    S0 = pace_synth.random_state(len(heads), w.d_v, w.d_k, seed=seed).numpy()
+    state, _ = orc.PoolState.from_fp32(S0, [bits[h] for _, h in heads], w.axis)
+    toks = []
+    for t in range(w.P):
+        inp = pace_synth.token_inputs(sub, t, seed=seed)
+        toks.append({k: v.reshape(len(heads), -1).double().numpy().squeeze(-1) if v.dim() == 2
+                     else v.reshape(len(heads), -1).double().numpy() for k, v in inp.items()})
+    t0 = time.perf_counter()
+    orc.period_reference(state, toks, w.P)
+    dt = time.perf_counter() - t0
+    units = len(heads) * w.P
+    return {"value": units / dt, "unit": "head-tokens/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{slots} slots x {w.H} heads ({len(heads)} heads), one period of P={w.P} "
+                      f"tokens plus its commit, fp64 numpy, {dt:.1f} s"}
+
+
+def alg_bytes(w, bits, n: int):
+    """Algorithmic DRAM bytes of one decode launch at buffer position n
+    (1..P) and of one commit launch (every head commits)."""
+    import bit_recurrent_state_pace_b200 as pace
+    rec = [pace.pace_pool_bytes(1, 1, w.d_k, w.d_v, w.P, 0, 0, [b])[0] for b in bits]
+    esz = 2 if w.io_dtype == "bf16" else 4
+    row = (w.d_k + w.d_v + 2) * esz            # buffered k, v, alpha, beta
+    inp = (2 * w.d_k + w.d_v + 2) * esz        # q, k, v, alpha, beta of the token
+    per_head = inp + (n - 1) * row + row + 4 * w.d_v + 8   # + buffer row write + o + fill r/w
+    decode = w.B * sum(rec) + w.B * w.H * per_head
+    commit = 2 * w.B * sum(rec) + w.B * w.H * (w.P * row + 8)
+    return decode, commit
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    import pace_synth
+    w = pace_synth.workload(args.workload)
+    if args.period:
+        w = w.replace(P=args.period)
+    bits = pace_synth.head_bits(w, args.seed)
+    samples = []
+    # each step: one whole sequence (all H heads) for one period, so that the
+    # default --steps/--warmup run stays within a few minutes of CPU time
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, bits, 1, args.seed)
+    for _ in range(args.steps):
+        samples.append(oracle_sample_rate(w, bits, 1, args.seed))
+    val = statistics.median(s["value"] for s in samples)
+    base = samples[0]
+    per_step_ms = 1000.0 * w.B * w.H * w.P / val
+    line = {
+        "impl": "reference", "metric": "decode head-tokens/s (B x H heads, 4-bit state, P=%d)" % w.P,
+        "value": val, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, bits),
+        "cpu_baseline": dict(base, value=val),
+        "e2e": {"value": val, "unit": "head-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, bits):
+    n8 = sum(1 for b in bits if b == 8)
+    return {"workload": f"{w.name}: B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} P={w.P} "
+                        f"{n8}/{w.H} INT8 heads, {w.axis} scales, {w.io_dtype} io",
+            "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "P": w.P, "int8_heads": n8,
+            "scale_axis": w.axis, "io_dtype": w.io_dtype, "state_dtype": "int4/int8 codes + fp16 scales",
+            "l2": "state pool larger than L2 (no flush needed)", "prefill_tokens": w.warmup}
+
+
+def run_pace(args, rank: int, world: int):
+    import torch
+    import bit_recurrent_state_pace_b200 as pace
+    import pace_synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = pace_synth.workload(args.workload)
+    if args.period:
+        w = w.replace(P=args.period)
+    if args.prefill is not None:
+        w = w.replace(warmup=args.prefill)
+    bits = pace_synth.head_bits(w, args.seed)
+    BH, P = w.B * w.H, w.P
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = oracle_sample_rate(w, bits, args.cpu_sample_slots, args.seed)
+
+    # ---- state: unquantised fp32 prefill, then encode into the pool
+    pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, P, bits, axis=w.axis, io=w.io_dtype, device=dev)
+    S = torch.zeros(BH, w.d_v, w.d_k, dtype=torch.float32, device=dev)
+    for t in range(w.warmup):
+        inp = pace_synth.token_inputs(w, t, seed=args.seed + rank, device=dev, phase="warmup")
+        pace.pace_gdn_step_f32(S, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                               pool.io, None, BH, w.d_k, w.d_v)
+    pool.load(S)
+    S_bf16 = None if args.no_compare else S.to(torch.bfloat16).view(torch.int16)
+    del S
+    torch.cuda.synchronize()
+
+    toks = [pace_synth.token_inputs(w, t, seed=args.seed + rank, device=dev) for t in range(P)]
+    outs = [torch.empty(w.B, w.H, w.d_v, dtype=torch.float32, device=dev) for _ in range(P)]
+
+    def period(ev=None):
+        for n in range(P):
+            x = toks[n]
+            if ev is not None:
+                ev[n][0].record(stream)
+            pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n], sp)
+            if ev is not None:
+                ev[n][1].record(stream)
+        if ev is not None:
+            ev[P][0].record(stream)
+        pace.pace_commit_period(pool.handle, sp)
+        if ev is not None:
+            ev[P][1].record(stream)
+
+    for _ in range(args.warmup):
+        period()
+    assert pool.status() == 0, "device status flags set during warm-up"
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [[(mk(), mk()) for _ in range(P + 1)] for _ in range(args.steps)]
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    if not gpu_uuid.startswith("GPU-"):
+        gpu_uuid = "GPU-" + gpu_uuid
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_uuid)
+    time.sleep(0.2)
+    t_start, t_end = mk(), mk()
+    t_start.record(stream)
+    for s in range(args.steps):
+        period(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    status = pool.status()
+
+    dec_ms = [[evs[s][n][0].elapsed_time(evs[s][n][1]) for s in range(args.steps)] for n in range(P)]
+    com_ms = [evs[s][P][0].elapsed_time(evs[s][P][1]) for s in range(args.steps)]
+    dec_bytes = [alg_bytes(w, bits, n + 1)[0] for n in range(P)]
+    com_bytes = alg_bytes(w, bits, P)[1]
+    dec_avg_ms = statistics.mean(statistics.mean(x) for x in dec_ms)
+    dec_avg_bytes = statistics.mean(dec_bytes)
+    com_avg_ms = statistics.mean(com_ms)
+    hbm, peak_kind = measured_peaks()
+    dec_gbs = dec_avg_bytes / (dec_avg_ms * 1e-3) / 1e9
+    com_gbs = com_bytes / (com_avg_ms * 1e-3) / 1e9
+    digest = kernel_source_digest()
+    dominant = "decode_step" if dec_avg_ms * P >= com_avg_ms else "commit"
+    if dominant == "decode_step":
+        ach, traffic = dec_gbs, ncu_traffic("decode_step", digest)
+    else:
+        ach, traffic = com_gbs, ncu_traffic("commit", digest)
+
+    units = BH * P * args.steps * world
+    value = units / (elapsed_ms * 1e-3)
+
+    # ---- bf16-state comparison path (unquantised, same shape)
+    compare = None
+    if S_bf16 is not None:
+        for _ in range(2):
+            x = toks[0]
+            pace.pace_gdn_step_bf16(S_bf16, x["q"], x["k"], x["v"], x["alpha"], x["beta"], pool.io,
+                                    outs[0], BH, w.d_k, w.d_v, sp)
+        ntok = 2 * P
+        a, b = mk(), mk()
+        a.record(stream)
+        for t in range(ntok):
+            x = toks[t % P]
+            pace.pace_gdn_step_bf16(S_bf16, x["q"], x["k"], x["v"], x["alpha"], x["beta"], pool.io,
+                                    outs[t % P], BH, w.d_k, w.d_v, sp)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / ntok
+        esz = 2 if w.io_dtype == "bf16" else 4
+        bbytes = BH * (2 * w.d_v * w.d_k * 2 + (2 * w.d_k + w.d_v + 2) * esz + 4 * w.d_v)
+        compare = {"bf16_state": {"value": BH / (ms * 1e-3), "unit": "head-tokens/s",
+                                  "ms_per_token": ms, "achieved_gbs": bbytes / (ms * 1e-3) / 1e9,
+                                  "state_bytes": BH * w.d_v * w.d_k * 2},
+                   "pace_state_bytes": int(pool.state.numel()),
+                   "pace_ms_per_token": elapsed_ms / world / (args.steps * P) if world == 1 else None}
+        del S_bf16
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, pace, pool, w, toks, outs, stream, world, dev)
+
+    if rank == 0:
+        line = {
+            "metric": "decode head-tokens/s (B x H heads, 4-bit state, P=%d)" % P,
+            "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": dict(workload_config(w, bits), parallelism=f"{world} independent pools (no collective)",
+                           seq_tokens_per_s=value / w.H),
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                         "frac": ach / hbm, "traffic": traffic, "kernel": dominant,
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6.65 TB/s"},
+            "kernels": {
+                "decode_step": {"avg_ms": dec_avg_ms, "alg_bytes_per_launch": dec_avg_bytes,
+                                "achieved_gbs": dec_gbs, "frac_of_peak": dec_gbs / hbm,
+                                "ms_by_fill": [statistics.mean(x) for x in dec_ms]},
+                "commit": {"avg_ms": com_avg_ms, "alg_bytes_per_launch": com_bytes,
+                           "achieved_gbs": com_gbs, "frac_of_peak": com_gbs / hbm},
+                "source_digest": digest,
+            },
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": args.steps * (P + 1),
+            "device_status": status,
+            "comparison": compare,
+            "cpu_baseline": cpu_base,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev):
+    """Same metric through the public API: every step copies its P tokens'
+    inputs host->device from pinned memory and reads every output back."""
+    import torch
+    P = w.P
+    host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in toks]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(v.numel() * v.element_size() for t in host_in for v in t.values())
+    d2h = sum(o.numel() * o.element_size() for o in host_out)
+    sp = stream.cuda_stream
+
+    def step():
+        for n in range(P):
+            for k, v in host_in[n].items():
+                toks[n][k].copy_(v, non_blocking=True)
+            x = toks[n]
+            pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n], sp)
+            host_out[n].copy_(outs[n], non_blocking=True)
+        pace.pace_commit_period(pool.handle, sp)
+
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    units = w.B * w.H * P * args.e2e_steps * world
+    return {"value": units / (ms * 1e-3), "unit": "head-tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, dev):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, rank, world)
+        return
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_pace(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,281 @@
+"""Python binding of libpace (PACE periodic low-bit recurrent-state decode).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of ``libpace.so``.  PyTorch supplies device memory and streams.
+The functions keep the C names of ``include/pace.h``; ``PacePool`` is a
+convenience owner of the three device regions a pool needs.
+
+Importing this package loads ``libpace.so`` from this directory and raises
+``ImportError`` if it is missing (build it with
+``python -m bit_recurrent_state_pace_b200.build``); there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "PaceError", "lib", "LIB_PATH",
+    "PACE_SCALE_COL", "PACE_SCALE_ROW", "PACE_IO_BF16", "PACE_IO_F32",
+    "PACE_FLAG_NONFINITE", "PACE_FLAG_SCALE_OVERFLOW", "PACE_FLAG_BUFFER_FULL", "PACE_FLAG_TIMEOUT",
+    "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
+    "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
+    "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
+    "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
+    "PacePool",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpace.so")
+
+PACE_SCALE_COL, PACE_SCALE_ROW = 0, 1
+PACE_IO_BF16, PACE_IO_F32 = 0, 1
+PACE_FLAG_NONFINITE = 0x1
+PACE_FLAG_SCALE_OVERFLOW = 0x2
+PACE_FLAG_BUFFER_FULL = 0x4
+PACE_FLAG_TIMEOUT = 0x8
+PACE_OK, PACE_ERR_DEVICE_FLAGS = 0, 4
+
+
+class PaceError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {_status_name(status)} ({status})")
+        self.status = status
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("num_slots", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("period", ctypes.c_int32),
+                ("scale_axis", ctypes.c_int32), ("io_dtype", ctypes.c_int32),
+                ("head_bits", ctypes.POINTER(ctypes.c_uint8))]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libpace.so not found at {LIB_PATH}: build it with "
+                          "`python -m bit_recurrent_state_pace_b200.build` (there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, S, I32, I64, U32p, U16p, F32p = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32,
+                                        ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p)
+    Sp = ctypes.POINTER(ctypes.c_size_t)
+    sig = {
+        "pace_pool_bytes": [ctypes.POINTER(_Desc), Sp, Sp, Sp],
+        "pace_init_pool": [ctypes.POINTER(_Desc), P, P, P, P, ctypes.POINTER(ctypes.c_void_p)],
+        "pace_pool_layout": [P, I32, Sp, Sp, Sp],
+        "pace_pool_load": [P, F32p, P],
+        "pace_pool_export": [P, F32p, P],
+        "pace_decode_step": [P, P, P, P, P, P, F32p, P],
+        "pace_commit_period": [P, P],
+        "pace_quantize": [F32p, I64, I32, I32, I32, I32, P, U16p, U32p, P],
+        "pace_dequantize": [P, U16p, I64, I32, I32, I32, I32, F32p, P],
+        "pace_pool_status": [P, P, ctypes.POINTER(ctypes.c_uint32)],
+        "pace_pool_clear_status": [P, P],
+        "pace_gdn_step_f32": [F32p, P, P, P, P, P, I32, F32p, I64, I32, I32, P],
+        "pace_gdn_step_bf16": [U16p, P, P, P, P, P, I32, F32p, I64, I32, I32, P],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.pace_destroy_pool.argtypes = [P]
+    L.pace_destroy_pool.restype = None
+    L.pace_status_string.argtypes = [ctypes.c_int]
+    L.pace_status_string.restype = ctypes.c_char_p
+    L.pace_version.argtypes = []
+    L.pace_version.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def _status_name(s: int) -> str:
+    return lib.pace_status_string(int(s)).decode()
+
+
+def _check(fn: str, status: int, ok=(PACE_OK,)) -> int:
+    if status not in ok:
+        raise PaceError(fn, status)
+    return status
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libpace takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libpace takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _desc(B, H, d_k, d_v, P, axis, io, head_bits) -> Tuple[_Desc, ctypes.Array]:
+    vals = [int(b) for b in head_bits]
+    bits_arr = (ctypes.c_uint8 * max(len(vals), 1))(*vals)
+    d = _Desc(B, H, d_k, d_v, P, axis, io, ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_uint8)))
+    return d, bits_arr
+
+
+# ---------------------------------------------------------------- C names
+
+def pace_pool_bytes(B, H, d_k, d_v, P, axis, io, head_bits) -> Tuple[int, int, int]:
+    d, keep = _desc(B, H, d_k, d_v, P, axis, io, head_bits)
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check("pace_pool_bytes", lib.pace_pool_bytes(ctypes.byref(d), ctypes.byref(a), ctypes.byref(b),
+                                                   ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def pace_init_pool(B, H, d_k, d_v, P, axis, io, head_bits, state, buffer, aux, stream=None) -> int:
+    d, keep = _desc(B, H, d_k, d_v, P, axis, io, head_bits)
+    out = ctypes.c_void_p()
+    _check("pace_init_pool", lib.pace_init_pool(ctypes.byref(d), _ptr(state), _ptr(buffer), _ptr(aux),
+                                                 _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def pace_destroy_pool(handle: int) -> None:
+    lib.pace_destroy_pool(handle)
+
+
+def pace_pool_layout(handle: int, head: int) -> Tuple[int, int, int]:
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check("pace_pool_layout", lib.pace_pool_layout(handle, head, ctypes.byref(a), ctypes.byref(b),
+                                                     ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def pace_pool_load(handle: int, S: torch.Tensor, stream=None) -> None:
+    _check("pace_pool_load", lib.pace_pool_load(handle, _ptr(S), _stream(stream)))
+
+
+def pace_pool_export(handle: int, S: torch.Tensor, stream=None) -> None:
+    _check("pace_pool_export", lib.pace_pool_export(handle, _ptr(S), _stream(stream)))
+
+
+def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
+    _check("pace_decode_step", lib.pace_decode_step(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                                     _ptr(beta), _ptr(o), _stream(stream)))
+
+
+def pace_commit_period(handle: int, stream=None) -> None:
+    _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_quantize(S, n_mats, d_k, d_v, bits, axis, codes, scales, flags=None, stream=None) -> None:
+    _check("pace_quantize", lib.pace_quantize(_ptr(S), n_mats, d_k, d_v, bits, axis, _ptr(codes),
+                                               _ptr(scales), _ptr(flags), _stream(stream)))
+
+
+def pace_dequantize(codes, scales, n_mats, d_k, d_v, bits, axis, S, stream=None) -> None:
+    _check("pace_dequantize", lib.pace_dequantize(_ptr(codes), _ptr(scales), n_mats, d_k, d_v, bits,
+                                                   axis, _ptr(S), _stream(stream)))
+
+
+def pace_pool_status(handle: int, stream=None) -> int:
+    f = ctypes.c_uint32()
+    _check("pace_pool_status", lib.pace_pool_status(handle, _stream(stream), ctypes.byref(f)),
+           ok=(PACE_OK, PACE_ERR_DEVICE_FLAGS))
+    return f.value
+
+
+def pace_pool_clear_status(handle: int, stream=None) -> None:
+    _check("pace_pool_clear_status", lib.pace_pool_clear_status(handle, _stream(stream)))
+
+
+def pace_gdn_step_f32(S, q, k, v, alpha, beta, io, o, n, d_k, d_v, stream=None) -> None:
+    _check("pace_gdn_step_f32", lib.pace_gdn_step_f32(_ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                                       _ptr(beta), io, _ptr(o), n, d_k, d_v,
+                                                       _stream(stream)))
+
+
+def pace_gdn_step_bf16(S, q, k, v, alpha, beta, io, o, n, d_k, d_v, stream=None) -> None:
+    _check("pace_gdn_step_bf16", lib.pace_gdn_step_bf16(_ptr(S), _ptr(q), _ptr(k), _ptr(v),
+                                                         _ptr(alpha), _ptr(beta), io, _ptr(o), n,
+                                                         d_k, d_v, _stream(stream)))
+
+
+def pace_status_string(status: int) -> str:
+    return _status_name(status)
+
+
+def pace_version() -> str:
+    return lib.pace_version().decode()
+
+
+# ---------------------------------------------------------------- pool owner
+
+class PacePool:
+    """Allocates a pool's three device regions with torch and binds them.
+
+    ``state``, ``buffer`` and ``aux`` are uint8 device tensors; their layout is
+    the one documented in ``include/pace.h``.
+    """
+
+    def __init__(self, B: int, H: int, d_k: int, d_v: int, P: int, head_bits: Sequence[int],
+                 axis: str = "col", io: str = "bf16", device="cuda", stream=None):
+        self.B, self.H, self.d_k, self.d_v, self.P = B, H, d_k, d_v, P
+        self.head_bits = [int(b) for b in head_bits]
+        self.axis = PACE_SCALE_COL if axis == "col" else PACE_SCALE_ROW
+        self.io = PACE_IO_BF16 if io == "bf16" else PACE_IO_F32
+        self.io_torch = torch.bfloat16 if io == "bf16" else torch.float32
+        sb, bb, ab = pace_pool_bytes(B, H, d_k, d_v, P, self.axis, self.io, self.head_bits)
+        self.state = torch.empty(sb, dtype=torch.uint8, device=device)
+        self.buffer = torch.zeros(bb, dtype=torch.uint8, device=device)
+        self.aux = torch.empty(ab, dtype=torch.uint8, device=device)
+        self.handle = pace_init_pool(B, H, d_k, d_v, P, self.axis, self.io, self.head_bits,
+                                     self.state, self.buffer, self.aux, stream)
+        self.slot_stride = pace_pool_layout(self.handle, 0)[2]
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            pace_destroy_pool(h)
+            self.handle = None
+
+    # layout helpers -----------------------------------------------------
+    def record(self, b: int, h: int) -> torch.Tensor:
+        """View of head (b, h)'s record (codes then fp16 scales) in the state region."""
+        off, nbytes, stride = pace_pool_layout(self.handle, h)
+        start = b * stride + off
+        return self.state[start:start + nbytes]
+
+    def fill(self) -> torch.Tensor:
+        return self.aux[: 4 * self.B * self.H].view(torch.int32).view(self.B, self.H)
+
+    # calls ----------------------------------------------------------------
+    def load(self, S: torch.Tensor, stream=None) -> None:
+        pace_pool_load(self.handle, S, stream)
+
+    def export(self, S: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        if S is None:
+            S = torch.empty(self.B, self.H, self.d_v, self.d_k, dtype=torch.float32,
+                            device=self.state.device)
+        pace_pool_export(self.handle, S, stream)
+        return S
+
+    def decode_step(self, q, k, v, alpha, beta, o=None, stream=None) -> torch.Tensor:
+        if o is None:
+            o = torch.empty(self.B, self.H, self.d_v, dtype=torch.float32, device=self.state.device)
+        pace_decode_step(self.handle, q, k, v, alpha, beta, o, stream)
+        return o
+
+    def commit_period(self, stream=None) -> None:
+        pace_commit_period(self.handle, stream)
+
+    def status(self, stream=None) -> int:
+        return pace_pool_status(self.handle, stream)
+
+    def clear_status(self, stream=None) -> None:
+        pace_pool_clear_status(self.handle, stream)

@@ -1,0 +1,78 @@
+// Internal declarations shared by the libpace CUDA sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/pace.h"
+
+#define PACE_MAX_HEADS 256
+#define PACE_MAX_PERIOD 16
+#define PACE_MAX_D 128
+
+namespace pace {
+
+// Everything a pool kernel needs, passed by value as a kernel parameter.
+struct PoolDev {
+  int32_t B, H, d_k, d_v, P, axis, io;
+  int32_t n_groups;           // scale groups per head: d_k (COL) or d_v (ROW)
+  uint64_t slot_stride;       // bytes per slot in the state region
+  uint8_t* state;             // [B][slot_stride]
+  uint8_t* kv;                // [B][H][P][d_k + d_v] io elements
+  uint8_t* ab;                // [B][H][P][2] io elements
+  int32_t* fill;              // [B][H]
+  uint32_t* flags;            // status word
+  uint32_t rec_off[PACE_MAX_HEADS];   // record offset of head h inside a slot
+  uint8_t bits[PACE_MAX_HEADS];       // 4 or 8
+};
+
+__host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline size_t code_bytes(int d_k, int d_v, int bits) {
+  return (size_t)d_v * (size_t)d_k * (size_t)bits / 8;
+}
+
+__host__ __device__ inline size_t record_bytes(int d_k, int d_v, int bits, int n_groups) {
+  return round_up(code_bytes(d_k, d_v, bits) + 2 * (size_t)n_groups, 16);
+}
+
+__host__ __device__ inline int io_size(int io) { return io == PACE_IO_BF16 ? 2 : 4; }
+
+// Load element `idx` of an io-dtype array as fp32.
+__device__ __forceinline__ float load_io(const void* p, size_t idx, int io) {
+  if (io == PACE_IO_BF16) {
+    uint16_t b = reinterpret_cast<const uint16_t*>(p)[idx];
+    return __uint_as_float(((uint32_t)b) << 16);
+  }
+  return reinterpret_cast<const float*>(p)[idx];
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits_rn(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// Host-side launchers (defined in the .cu files, called by pool.cu).
+cudaError_t launch_quantize(const float* S, int64_t n, int d_k, int d_v, int bits, int axis,
+                            uint8_t* codes, uint16_t* scales, uint32_t* flags, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint16_t* scales, int64_t n, int d_k,
+                              int d_v, int bits, int axis, float* S, cudaStream_t st);
+cudaError_t launch_pool_load(const PoolDev& p, const float* S, cudaStream_t st);
+cudaError_t launch_pool_export(const PoolDev& p, float* S, cudaStream_t st);
+cudaError_t launch_decode_step(const PoolDev& p, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* beta, float* o, cudaStream_t st);
+cudaError_t launch_commit(const PoolDev& p, cudaStream_t st);
+cudaError_t launch_gdn_step_f32(float* S, const void* q, const void* k, const void* v,
+                                const void* alpha, const void* beta, int io, float* o, int64_t n,
+                                int d_k, int d_v, cudaStream_t st);
+cudaError_t launch_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const void* v,
+                                 const void* alpha, const void* beta, int io, float* o, int64_t n,
+                                 int d_k, int d_v, cudaStream_t st);
+
+}  // namespace pace

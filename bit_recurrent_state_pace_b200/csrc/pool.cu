@@ -1,0 +1,264 @@
+// Host side of the libpace C ABI: argument validation, pool layout, launches.
+#include <new>
+#include <string.h>
+
+#include "pace_internal.cuh"
+
+struct pace_pool {
+  pace::PoolDev dev;
+  pace_pool_desc desc;
+  size_t state_bytes, buffer_bytes, aux_bytes, kv_bytes;
+  size_t rec_bytes[PACE_MAX_HEADS];
+};
+
+namespace {
+
+using pace::round_up;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline pace_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return PACE_OK;
+  (void)cudaGetLastError();  // clear a non-sticky error so later calls start clean
+  return PACE_ERR_CUDA;
+}
+
+inline bool mul_ok(size_t a, size_t b, size_t* out) {
+  if (a != 0 && b > SIZE_MAX / a) return false;
+  *out = a * b;
+  return true;
+}
+
+struct Layout {
+  size_t slot_stride;
+  size_t rec_off[PACE_MAX_HEADS];
+  size_t rec_bytes[PACE_MAX_HEADS];
+  size_t state_bytes, kv_bytes, buffer_bytes, aux_bytes;
+  int n_groups;
+};
+
+pace_status check_desc(const pace_pool_desc* d) {
+  if (!d) return PACE_ERR_INVALID_ARG;
+  if (d->num_slots < 1 || d->num_heads < 1 || d->num_heads > PACE_MAX_HEADS) return PACE_ERR_INVALID_ARG;
+  if (d->period < 1 || d->period > PACE_MAX_PERIOD) return PACE_ERR_INVALID_ARG;
+  if (d->scale_axis != PACE_SCALE_COL && d->scale_axis != PACE_SCALE_ROW) return PACE_ERR_INVALID_ARG;
+  if (d->io_dtype != PACE_IO_BF16 && d->io_dtype != PACE_IO_F32) return PACE_ERR_INVALID_ARG;
+  if (!d->head_bits) return PACE_ERR_INVALID_ARG;
+  for (int h = 0; h < d->num_heads; ++h)
+    if (d->head_bits[h] != 4 && d->head_bits[h] != 8) return PACE_ERR_INVALID_ARG;
+  if (d->d_k < 1 || d->d_v < 1) return PACE_ERR_INVALID_ARG;
+  if (d->d_k != d->d_v) return PACE_ERR_UNSUPPORTED;
+  if (d->d_k != 32 && d->d_k != 64 && d->d_k != 128) return PACE_ERR_UNSUPPORTED;
+  return PACE_OK;
+}
+
+pace_status compute_layout(const pace_pool_desc* d, Layout* L) {
+  pace_status st = check_desc(d);
+  if (st != PACE_OK) return st;
+  L->n_groups = d->scale_axis == PACE_SCALE_COL ? d->d_k : d->d_v;
+  size_t off = 0;
+  for (int h = 0; h < d->num_heads; ++h) {
+    L->rec_off[h] = off;
+    L->rec_bytes[h] = pace::record_bytes(d->d_k, d->d_v, d->head_bits[h], L->n_groups);
+    off += L->rec_bytes[h];
+  }
+  L->slot_stride = round_up(off, 16);
+  if (!mul_ok(L->slot_stride, (size_t)d->num_slots, &L->state_bytes)) return PACE_ERR_INVALID_ARG;
+  const size_t esz = (size_t)pace::io_size(d->io_dtype);
+  size_t heads = 0, rows = 0, kv = 0, ab = 0;
+  if (!mul_ok((size_t)d->num_slots, (size_t)d->num_heads, &heads)) return PACE_ERR_INVALID_ARG;
+  if (!mul_ok(heads, (size_t)d->period, &rows)) return PACE_ERR_INVALID_ARG;
+  if (!mul_ok(rows, (size_t)(d->d_k + d->d_v) * esz, &kv)) return PACE_ERR_INVALID_ARG;
+  if (!mul_ok(rows, 2 * esz, &ab)) return PACE_ERR_INVALID_ARG;
+  L->kv_bytes = round_up(kv, 256);
+  L->buffer_bytes = L->kv_bytes + round_up(ab, 256);
+  L->aux_bytes = round_up(4 * heads, 256) + 256;
+  if (heads > 0x7fffffffULL) return PACE_ERR_UNSUPPORTED;
+  return PACE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pace_status_string(pace_status s) {
+  switch (s) {
+    case PACE_OK: return "PACE_OK";
+    case PACE_ERR_INVALID_ARG: return "PACE_ERR_INVALID_ARG";
+    case PACE_ERR_UNSUPPORTED: return "PACE_ERR_UNSUPPORTED";
+    case PACE_ERR_CUDA: return "PACE_ERR_CUDA";
+    case PACE_ERR_DEVICE_FLAGS: return "PACE_ERR_DEVICE_FLAGS";
+  }
+  return "PACE_ERR_UNKNOWN";
+}
+
+const char* pace_version(void) { return "0.1.0"; }
+
+pace_status pace_pool_bytes(const pace_pool_desc* desc, size_t* state_bytes, size_t* buffer_bytes,
+                            size_t* aux_bytes) {
+  if (!state_bytes || !buffer_bytes || !aux_bytes) return PACE_ERR_INVALID_ARG;
+  Layout L;
+  pace_status st = compute_layout(desc, &L);
+  if (st != PACE_OK) return st;
+  *state_bytes = L.state_bytes;
+  *buffer_bytes = L.buffer_bytes;
+  *aux_bytes = L.aux_bytes;
+  return PACE_OK;
+}
+
+pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_buffer, void* d_aux,
+                           void* stream, pace_pool** out) {
+  if (!out) return PACE_ERR_INVALID_ARG;
+  *out = nullptr;
+  Layout L;
+  pace_status st = compute_layout(desc, &L);
+  if (st != PACE_OK) return st;
+  if (!d_state || !d_buffer || !d_aux) return PACE_ERR_INVALID_ARG;
+  if (!aligned(d_state, 256) || !aligned(d_buffer, 256) || !aligned(d_aux, 256)) return PACE_ERR_INVALID_ARG;
+  pace_pool* p = new (std::nothrow) pace_pool;
+  if (!p) return PACE_ERR_INVALID_ARG;
+  memset(p, 0, sizeof(*p));
+  p->desc = *desc;
+  p->desc.head_bits = nullptr;
+  p->state_bytes = L.state_bytes;
+  p->buffer_bytes = L.buffer_bytes;
+  p->aux_bytes = L.aux_bytes;
+  p->kv_bytes = L.kv_bytes;
+  pace::PoolDev& dv = p->dev;
+  dv.B = desc->num_slots;
+  dv.H = desc->num_heads;
+  dv.d_k = desc->d_k;
+  dv.d_v = desc->d_v;
+  dv.P = desc->period;
+  dv.axis = desc->scale_axis;
+  dv.io = desc->io_dtype;
+  dv.n_groups = L.n_groups;
+  dv.slot_stride = L.slot_stride;
+  dv.state = static_cast<uint8_t*>(d_state);
+  dv.kv = static_cast<uint8_t*>(d_buffer);
+  dv.ab = static_cast<uint8_t*>(d_buffer) + L.kv_bytes;
+  dv.fill = static_cast<int32_t*>(d_aux);
+  dv.flags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(d_aux) + L.aux_bytes - 256);
+  for (int h = 0; h < desc->num_heads; ++h) {
+    dv.rec_off[h] = (uint32_t)L.rec_off[h];
+    dv.bits[h] = desc->head_bits[h];
+    p->rec_bytes[h] = L.rec_bytes[h];
+  }
+  cudaError_t e = cudaMemsetAsync(d_aux, 0, L.aux_bytes, as_stream(stream));
+  if (e != cudaSuccess) {
+    delete p;
+    return from_cuda(e);
+  }
+  *out = p;
+  return PACE_OK;
+}
+
+void pace_destroy_pool(pace_pool* pool) { delete pool; }
+
+pace_status pace_pool_layout(const pace_pool* pool, int32_t head, size_t* record_offset,
+                             size_t* record_bytes, size_t* slot_stride) {
+  if (!pool || !record_offset || !record_bytes || !slot_stride) return PACE_ERR_INVALID_ARG;
+  if (head < 0 || head >= pool->dev.H) return PACE_ERR_INVALID_ARG;
+  *record_offset = pool->dev.rec_off[head];
+  *record_bytes = pool->rec_bytes[head];
+  *slot_stride = pool->dev.slot_stride;
+  return PACE_OK;
+}
+
+pace_status pace_pool_load(pace_pool* pool, const float* S, void* stream) {
+  if (!pool || !S || !aligned(S, 16)) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_pool_load(pool->dev, S, as_stream(stream)));
+}
+
+pace_status pace_pool_export(pace_pool* pool, float* S, void* stream) {
+  if (!pool || !S || !aligned(S, 16)) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_pool_export(pool->dev, S, as_stream(stream)));
+}
+
+pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, const void* v,
+                             const void* alpha, const void* beta, float* o, void* stream) {
+  if (!pool || !q || !k || !v || !alpha || !beta || !o) return PACE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return PACE_ERR_INVALID_ARG;
+  if (!aligned(alpha, 4) || !aligned(beta, 4)) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_decode_step(pool->dev, q, k, v, alpha, beta, o, as_stream(stream)));
+}
+
+pace_status pace_commit_period(pace_pool* pool, void* stream) {
+  if (!pool) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_commit(pool->dev, as_stream(stream)));
+}
+
+pace_status pace_quantize(const float* S, int64_t n_mats, int32_t d_k, int32_t d_v, int32_t bits,
+                          int32_t scale_axis, void* codes, uint16_t* scales, uint32_t* d_flags,
+                          void* stream) {
+  if (n_mats < 0 || n_mats > 0x7fffffffLL) return PACE_ERR_INVALID_ARG;
+  if (d_k < 2 || d_v < 2 || d_k > 256 || d_v > 256 || (d_k & 1)) return PACE_ERR_INVALID_ARG;
+  if (bits != 4 && bits != 8) return PACE_ERR_INVALID_ARG;
+  if (scale_axis != PACE_SCALE_COL && scale_axis != PACE_SCALE_ROW) return PACE_ERR_INVALID_ARG;
+  if (n_mats == 0) return PACE_OK;
+  if (!S || !codes || !scales) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_quantize(S, n_mats, d_k, d_v, bits, scale_axis,
+                                         static_cast<uint8_t*>(codes), scales, d_flags,
+                                         as_stream(stream)));
+}
+
+pace_status pace_dequantize(const void* codes, const uint16_t* scales, int64_t n_mats, int32_t d_k,
+                            int32_t d_v, int32_t bits, int32_t scale_axis, float* S, void* stream) {
+  if (n_mats < 0 || n_mats > 0x7fffffffLL) return PACE_ERR_INVALID_ARG;
+  if (d_k < 2 || d_v < 2 || d_k > 256 || d_v > 256 || (d_k & 1)) return PACE_ERR_INVALID_ARG;
+  if (bits != 4 && bits != 8) return PACE_ERR_INVALID_ARG;
+  if (scale_axis != PACE_SCALE_COL && scale_axis != PACE_SCALE_ROW) return PACE_ERR_INVALID_ARG;
+  if (n_mats == 0) return PACE_OK;
+  if (!S || !codes || !scales) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_dequantize(static_cast<const uint8_t*>(codes), scales, n_mats, d_k,
+                                           d_v, bits, scale_axis, S, as_stream(stream)));
+}
+
+pace_status pace_pool_status(pace_pool* pool, void* stream, uint32_t* flags) {
+  if (!pool || !flags) return PACE_ERR_INVALID_ARG;
+  uint32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, pool->dev.flags, sizeof(host), cudaMemcpyDeviceToHost,
+                                  as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return from_cuda(e);
+  *flags = host;
+  return host ? PACE_ERR_DEVICE_FLAGS : PACE_OK;
+}
+
+pace_status pace_pool_clear_status(pace_pool* pool, void* stream) {
+  if (!pool) return PACE_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(pool->dev.flags, 0, sizeof(uint32_t), as_stream(stream)));
+}
+
+static pace_status check_step_args(const void* S, const void* q, const void* k, const void* v,
+                                   const void* alpha, const void* beta, int32_t io, int64_t n,
+                                   int32_t d_k, int32_t d_v) {
+  if (n < 0 || n > 0x7fffffffLL) return PACE_ERR_INVALID_ARG;
+  if (io != PACE_IO_BF16 && io != PACE_IO_F32) return PACE_ERR_INVALID_ARG;
+  if (d_k != d_v) return PACE_ERR_UNSUPPORTED;
+  if (d_k != 32 && d_k != 64 && d_k != 128) return PACE_ERR_UNSUPPORTED;
+  if (n > 0 && (!S || !q || !k || !v || !alpha || !beta)) return PACE_ERR_INVALID_ARG;
+  return PACE_OK;
+}
+
+pace_status pace_gdn_step_f32(float* S, const void* q, const void* k, const void* v,
+                              const void* alpha, const void* beta, int32_t io_dtype, float* o,
+                              int64_t n, int32_t d_k, int32_t d_v, void* stream) {
+  pace_status st = check_step_args(S, q, k, v, alpha, beta, io_dtype, n, d_k, d_v);
+  if (st != PACE_OK) return st;
+  return from_cuda(pace::launch_gdn_step_f32(S, q, k, v, alpha, beta, io_dtype, o, n, d_k, d_v,
+                                             as_stream(stream)));
+}
+
+pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* beta, int32_t io_dtype, float* o,
+                               int64_t n, int32_t d_k, int32_t d_v, void* stream) {
+  pace_status st = check_step_args(S, q, k, v, alpha, beta, io_dtype, n, d_k, d_v);
+  if (st != PACE_OK) return st;
+  return from_cuda(pace::launch_gdn_step_bf16(S, q, k, v, alpha, beta, io_dtype, o, n, d_k, d_v,
+                                              as_stream(stream)));
+}
+
+}  // extern "C"

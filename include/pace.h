@@ -1,0 +1,209 @@
+/*
+ * pace.h -- C ABI of libpace: batched decode of a Gated DeltaNet linear-
+ * attention layer whose per-sequence recurrent state is stored as INT4 (or
+ * INT8 for chosen heads) with channel-aligned FP16 scales, rounded once per
+ * period of P tokens (PACE).
+ *
+ * Sources (page title, section):
+ *  [P2] "PACE: A New 4-Bit Recurrent State Quantization Method That Makes
+ *       Linear Attention Models More Memory-Efficient"
+ *  [P3] "低比特量化新突破：GGA+PW让线性注意力长文本生成更准更短"
+ *  [P4] "PACE: four-bit recurrent state by rounding less often"
+ *
+ * Conventions for every call:
+ *  - All tensors live in device memory allocated and owned by the caller
+ *    (e.g. by PyTorch); the library keeps pointers only, never allocates
+ *    device memory, and never frees caller memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream unless it says it
+ *    synchronises.
+ *  - Every call returns pace_status and never throws or aborts.  Argument
+ *    errors are detected on the host before any launch.  Conditions seen
+ *    on the device (non-finite values, a decode into a full buffer, a
+ *    bounded wait that gave up) set bits of the pool's device status word,
+ *    read with pace_pool_status().
+ *  - State matrices are S in R^{d_v x d_k}, stored row-major (row i = value
+ *    channel, column j = key channel), the state of the rule
+ *      S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t
+ *    (reading of the gate + delta rule described in [P3], section
+ *    "为什么低比特状态量化会“越写越错”").
+ */
+#ifndef PACE_H_
+#define PACE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PACE_OK = 0,
+  PACE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad enum, misaligned pointer */
+  PACE_ERR_UNSUPPORTED = 2,  /* a shape the kernels are not built for */
+  PACE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  PACE_ERR_DEVICE_FLAGS = 4  /* pace_pool_status found device status bits set */
+} pace_status;
+
+/* Device status bits (pace_pool_status, pace_quantize's d_flags). */
+#define PACE_FLAG_NONFINITE      0x1u  /* a scale group held a NaN/Inf: scale NaN, codes 0 */
+#define PACE_FLAG_SCALE_OVERFLOW 0x2u  /* amax/qmax exceeded fp16: scale clamped to 65504 */
+#define PACE_FLAG_BUFFER_FULL    0x4u  /* decode into a head whose buffer held P tokens:
+                                          that head's output row is NaN, nothing stored */
+#define PACE_FLAG_TIMEOUT        0x8u  /* a bounded wait inside a kernel gave up */
+
+/* Scale axis ([P2] "Channel-Aligned Encoding"; [P4] TL;DR (2)).
+ * COL: one scale per key channel j, shared by the d_v entries S[:, j].
+ * ROW: one scale per value channel i, shared by the d_k entries S[i, :]. */
+typedef enum { PACE_SCALE_COL = 0, PACE_SCALE_ROW = 1 } pace_scale_axis;
+
+/* Element type of q, k, v, alpha, beta and of the token buffer. */
+typedef enum { PACE_IO_BF16 = 0, PACE_IO_F32 = 1 } pace_io_dtype;
+
+typedef struct pace_pool pace_pool;  /* opaque, host-side */
+
+typedef struct {
+  int32_t num_slots;          /* B: sequences decoded together (>= 1) */
+  int32_t num_heads;          /* H: value heads (1..256) */
+  int32_t d_k, d_v;           /* head dims; supported: d_k == d_v in {32, 64, 128} */
+  int32_t period;             /* P: tokens per rounding period, 1..16 */
+  int32_t scale_axis;         /* pace_scale_axis */
+  int32_t io_dtype;           /* pace_io_dtype */
+  const uint8_t* head_bits;   /* host array [num_heads], each 4 or 8 ([P4] TL;DR (3)) */
+} pace_pool_desc;
+
+/*
+ * Memory a pool needs, in bytes (host-only query, no CUDA call).
+ *
+ * state  : B slots of `slot_stride` bytes.  Slot b holds every head's record
+ *          at the offset pace_pool_layout() reports.  A record is the codes,
+ *          d_v rows of d_k*bits/8 bytes (INT8: two's complement bytes; INT4:
+ *          two codes per byte, the even key index j in the low nibble, each
+ *          nibble the 4-bit two's complement of a code in [-7, 7]), followed
+ *          by the head's FP16 scales (d_k of them for COL, d_v for ROW), the
+ *          record padded to 16 bytes.
+ * buffer : the token buffer ([P2] "Periodic Rounding"; [P4] flowchart "Small
+ *          buffer, last few tokens"): region KV = [B][H][P][d_k + d_v]
+ *          io_dtype elements (row = k then v of one buffered token), then at
+ *          byte offset round_up(size(KV), 256) region AB = [B][H][P][2]
+ *          io_dtype elements (alpha, beta).  q is not stored: no later step
+ *          reads an old query.
+ * aux    : fill counters int32 [B][H] (tokens in each head's buffer), then at
+ *          byte offset round_up(4*B*H, 256) the uint32 status word.
+ * All three regions must be 256-byte aligned.
+ */
+pace_status pace_pool_bytes(const pace_pool_desc* desc, size_t* state_bytes,
+                            size_t* buffer_bytes, size_t* aux_bytes);
+
+/*
+ * Bind caller-owned device regions to a new pool.  Copies the descriptor
+ * (head_bits included), computes the record layout, and zeroes aux (all
+ * buffers empty, status clear) with cudaMemsetAsync on `stream`.  The state
+ * contents are the caller's (fill them with pace_pool_load or by writing
+ * records directly).  The regions must outlive the pool.
+ */
+pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_buffer,
+                           void* d_aux, void* stream, pace_pool** out);
+
+/* Release the host-side pool object (caller memory is untouched). NULL is a no-op. */
+void pace_destroy_pool(pace_pool* pool);
+
+/* Byte offset of head h's record inside a slot, its size, and the slot stride. */
+pace_status pace_pool_layout(const pace_pool* pool, int32_t head, size_t* record_offset,
+                             size_t* record_bytes, size_t* slot_stride);
+
+/*
+ * Encode S (device fp32 [B][H][d_v][d_k]) into every head's record with that
+ * head's bit width, and empty every buffer (fill = 0).  Same encoding as
+ * pace_quantize.
+ */
+pace_status pace_pool_load(pace_pool* pool, const float* S, void* stream);
+
+/* Decode every stored state to S (device fp32 [B][H][d_v][d_k]); buffered
+ * tokens are not applied. */
+pace_status pace_pool_export(pace_pool* pool, float* S, void* stream);
+
+/*
+ * One decode token for every head of every slot ([P2] "Periodic Rounding":
+ * tokens wait in a small buffer and the state is not rounded).
+ * q, k: [B][H][d_k]; v: [B][H][d_v]; alpha, beta: [B][H]; all io_dtype.
+ * o: fp32 [B][H][d_v].
+ * For each head with n-1 buffered tokens (n <= P): appends the token as row
+ * n-1 of the head's buffer and writes o_n = S_n q_n exactly in chunk form
+ * from the stored state S~0 (the decayed stored state applied to q_n plus
+ * the delta-rule correction of the n buffered tokens, fp32 accumulation),
+ * then sets fill = n.  The stored state is not modified.  A head whose buffer
+ * already holds P tokens is skipped (o row NaN, PACE_FLAG_BUFFER_FULL): call
+ * pace_commit_period after the step that fills the buffer.
+ */
+pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, const void* v,
+                             const void* alpha, const void* beta, float* o, void* stream);
+
+/*
+ * Period end ([P4] flowchart "every k tokens -> State update, chunked, high
+ * precision -> 4-bit encode, per-column scales"; 8-bit heads from TL;DR (3)).
+ * For every head whose buffer holds P tokens: dequantise the stored state,
+ * apply the P buffered tokens in one chunked (UT/WY) update in fp32, encode
+ * the result with fresh absmax scales at the head's bit width, write it back
+ * in place, and empty the buffer.  Heads with fewer than P tokens are left
+ * untouched, so slots may run at different phases.
+ */
+pace_status pace_commit_period(pace_pool* pool, void* stream);
+
+/*
+ * Encode n_mats fp32 matrices S [n_mats][d_v][d_k] (device) with one FP16
+ * scale per group ([P2] "Channel-Aligned Encoding"):
+ *   amax = max|x| (group); s32 = amax/qmax (fp32 divide, round to nearest);
+ *   s16 = fp16_rn(s32), raised to 2^-24 if amax > 0 and s16 == 0, clamped to
+ *   65504 (+ PACE_FLAG_SCALE_OVERFLOW) if it overflows;
+ *   code = clamp(rint_half_even(x / float(s16)), -qmax, qmax), fp32 divide;
+ *   all codes 0 if s16 == 0; a group holding NaN/Inf gets scale NaN (0x7E00),
+ *   codes 0 and PACE_FLAG_NONFINITE.
+ * qmax = 7 (bits 4) or 127 (bits 8).
+ * codes: [n_mats][d_v][d_k*bits/8] bytes, packed as in a pool record.
+ * scales: fp16 bits [n_mats][d_k] (COL) or [n_mats][d_v] (ROW).
+ * d_flags: optional device uint32 that receives the status bits (atomic OR).
+ * d_k, d_v: even, 2..256.
+ */
+pace_status pace_quantize(const float* S, int64_t n_mats, int32_t d_k, int32_t d_v,
+                          int32_t bits, int32_t scale_axis, void* codes, uint16_t* scales,
+                          uint32_t* d_flags, void* stream);
+
+/* Inverse of pace_quantize: S = float(code) * float(scale), exact in fp32. */
+pace_status pace_dequantize(const void* codes, const uint16_t* scales, int64_t n_mats,
+                            int32_t d_k, int32_t d_v, int32_t bits, int32_t scale_axis,
+                            float* S, void* stream);
+
+/* Synchronise `stream`, then read the pool's device status word into *flags.
+ * Returns PACE_ERR_DEVICE_FLAGS if any bit is set, PACE_OK otherwise. */
+pace_status pace_pool_status(pace_pool* pool, void* stream, uint32_t* flags);
+
+/* Clear the device status word (async on `stream`). */
+pace_status pace_pool_clear_status(pace_pool* pool, void* stream);
+
+/*
+ * Unquantised comparison paths (not PACE; used for the fp32 warm-up prefill,
+ * the drift reference trajectory and the bf16-state throughput comparison).
+ * One token of the rule above for n independent heads, state updated in
+ * place: S [n][d_v][d_k] fp32 (pace_gdn_step_f32) or bf16 bits
+ * (pace_gdn_step_bf16); q, k [n][d_k], v [n][d_v], alpha, beta [n] in
+ * io_dtype; o: fp32 [n][d_v] or NULL.  d_k == d_v in {32, 64, 128}.
+ */
+pace_status pace_gdn_step_f32(float* S, const void* q, const void* k, const void* v,
+                              const void* alpha, const void* beta, int32_t io_dtype,
+                              float* o, int64_t n, int32_t d_k, int32_t d_v, void* stream);
+pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* beta, int32_t io_dtype,
+                               float* o, int64_t n, int32_t d_k, int32_t d_v, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* pace_status_string(pace_status s);
+
+/* Library version, e.g. "0.1.0". */
+const char* pace_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PACE_H_ */

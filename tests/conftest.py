@@ -8,7 +8,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _ensure_library_built():
+    """Compile libpace.so in-tree if it is missing or older than its sources
+    (the build script runs without importing the package)."""
+    import subprocess
+    script = os.path.join(ROOT, "bit_recurrent_state_pace_b200", "build.py")
+    subprocess.run([sys.executable, script], check=True, stdout=subprocess.DEVNULL)
+
+
 def pytest_configure(config):
+    _ensure_library_built()
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: longer CPU test")
 
