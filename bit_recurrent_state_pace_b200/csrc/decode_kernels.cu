@@ -5,189 +5,376 @@
 // small buffer and the stored state is rounded only once per period; "PACE:
 // four-bit recurrent state by rounding less often", flowchart "New tokens ->
 // Small buffer".  The output of the n-th buffered token is exact in chunk
-// form from the stored state S~0 (the state is never materialised):
+// form from the stored state S~0 (the working state is never materialised):
 //
 //   o_n = S_n q_n = S~0 q^ + sum_s z_s v_s,   q^ = gamma_n q_n - sum_s z_s gamma_s k_s,
 //   z = diag(beta) (I + A)^{-T} w,  w_s = gamma_{n/s} (k_s . q_n),
 //   A[t][s] = beta_t gamma_{t/s} (k_t . k_s) for s < t,
 //
 // which follows from the UT/WY chunk form S_n = gamma_n S~0 + sum_s
-// gamma_{n/s} u_s k_s^T with U = (I + A)^{-1} diag(beta) (V - diag(gamma) X^T),
-// X = S~0 K^T, by moving (I + A)^{-1} onto the readout side: only one
-// state-sized product (S~0 q^) is needed per token.
-#include "encode.cuh"
+// gamma_{n/s} u_s k_s^T, U = (I + A)^{-1} diag(beta) (V - diag(gamma) X^T),
+// X = S~0 K^T, by moving (I + A)^{-1} to the readout side: one state-sized
+// product (S~0 q^) per token.
+//
+// Design (B200): one warp owns one head at a time (no block barriers); heads
+// are strided over a persistent grid.  The codes stream from HBM with
+// coalesced 128-bit non-allocating loads straight into the A-fragment
+// registers of mma.sync m16n8k16 (f16 codes exact, fp32 accumulation; the
+// right-hand side q^ is split hi + lo in f16), prefetched two 16-row blocks
+// ahead.  The small n x n chunk algebra runs lane-parallel over tokens with
+// warp shuffles; k.k dot products of earlier buffered tokens are cached in
+// the buffer's Gram region, so each step computes only the 2n-1 new ones.
+#include "frag.cuh"
 
 namespace pace {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kWarpsPerBlock = 8;
+constexpr int kThreads = kWarpsPerBlock * 32;
+constexpr unsigned FULL = 0xffffffffu;
 
-__global__ void __launch_bounds__(kThreads) decode_step_kernel(PoolDev p, const void* __restrict__ q,
-                                                               const void* __restrict__ k,
-                                                               const void* __restrict__ v,
-                                                               const void* __restrict__ alpha,
-                                                               const void* __restrict__ beta,
-                                                               float* __restrict__ o) {
-  __shared__ float Ks[PACE_MAX_PERIOD][PACE_MAX_D];
-  __shared__ float Vs[PACE_MAX_PERIOD][PACE_MAX_D];
-  __shared__ float qs[PACE_MAX_D], qhat[PACE_MAX_D], sc[PACE_MAX_D];
-  __shared__ float al[PACE_MAX_PERIOD], be[PACE_MAX_PERIOD], kq[PACE_MAX_PERIOD];
-  __shared__ float gram[PACE_MAX_PERIOD][PACE_MAX_PERIOD];
-  __shared__ float zv[PACE_MAX_PERIOD], zk[PACE_MAX_PERIOD], gamma_n;
-  __shared__ int n_sh;
+template <int D>
+struct alignas(16) WarpScratch {
+  __half bfrag[3][4][D / 16][4];   // [hi | lo | zero][lane group t][k-step][pos]
+  float y[D];                      // S~0 q^ by row, before the row scale
+};
 
-  const int head = blockIdx.x;
+// Lane L ends with the warp-wide sum of value index (L mod V).
+template <int V>
+__device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
+#pragma unroll
+  for (int c = V; c > 1; c >>= 1) {
+    const int o = c >> 1;
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int k = 0; k < c / 2; ++k) {
+      const float send = upper ? v[k] : v[k + c / 2];
+      const float keep = upper ? v[k + c / 2] : v[k];
+      v[k] = keep + __shfl_xor_sync(FULL, send, o);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int o = V; o < 32; o <<= 1) r += __shfl_xor_sync(FULL, r, o);
+  return r;
+}
+
+template <int D, bool BF16, int PMAX, int BITS>
+__device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, const void* __restrict__ q,
+                                            const void* __restrict__ k, const void* __restrict__ v,
+                                            const void* __restrict__ alpha,
+                                            const void* __restrict__ beta, float* __restrict__ o,
+                                            WarpScratch<D>& scr, int lane) {
+  constexpr int EPL = D / 32, RB = D / 16, KS = D / 16, PF = 2;
+  constexpr int ESZ = BF16 ? 2 : 4;
+  const int g = lane >> 2, t = lane & 3;
   const int h = head % p.H, b = head / p.H;
-  const int d_k = p.d_k, d_v = p.d_v, P = p.P, io = p.io, tid = threadIdx.x;
-  const int esz = io_size(io);
-  const int bits = p.bits[h];
-
-  if (tid == 0) {
-    const int n_prev = p.fill[head];
-    n_sh = (n_prev >= 0 && n_prev < P) ? n_prev + 1 : -1;
-    if (n_sh < 0) atomicOr(p.flags, PACE_FLAG_BUFFER_FULL);
-  }
-  __syncthreads();
-  const int n = n_sh;
-  if (n < 0) {
-    for (int i = tid; i < d_v; i += kThreads) o[(size_t)head * d_v + i] = __int_as_float(0x7fc00000);
-    return;
-  }
-
-  // current token -> shared memory and buffer row n-1 (raw io bits copied)
-  const size_t row_elems = (size_t)(d_k + d_v);
-  uint8_t* kv_head = p.kv + (size_t)head * P * row_elems * esz;
-  uint8_t* ab_head = p.ab + (size_t)head * P * 2 * esz;
-  for (int j = tid; j < d_k; j += kThreads) {
-    Ks[n - 1][j] = load_io(k, (size_t)head * d_k + j, io);
-    qs[j] = load_io(q, (size_t)head * d_k + j, io);
-    if (esz == 2)
-      reinterpret_cast<uint16_t*>(kv_head)[(n - 1) * row_elems + j] =
-          reinterpret_cast<const uint16_t*>(k)[(size_t)head * d_k + j];
-    else
-      reinterpret_cast<float*>(kv_head)[(n - 1) * row_elems + j] =
-          reinterpret_cast<const float*>(k)[(size_t)head * d_k + j];
-  }
-  for (int i = tid; i < d_v; i += kThreads) {
-    Vs[n - 1][i] = load_io(v, (size_t)head * d_v + i, io);
-    if (esz == 2)
-      reinterpret_cast<uint16_t*>(kv_head)[(n - 1) * row_elems + d_k + i] =
-          reinterpret_cast<const uint16_t*>(v)[(size_t)head * d_v + i];
-    else
-      reinterpret_cast<float*>(kv_head)[(n - 1) * row_elems + d_k + i] =
-          reinterpret_cast<const float*>(v)[(size_t)head * d_v + i];
-  }
-  if (tid == 0) {
-    al[n - 1] = load_io(alpha, head, io);
-    be[n - 1] = load_io(beta, head, io);
-    if (esz == 2) {
-      reinterpret_cast<uint16_t*>(ab_head)[(n - 1) * 2 + 0] = reinterpret_cast<const uint16_t*>(alpha)[head];
-      reinterpret_cast<uint16_t*>(ab_head)[(n - 1) * 2 + 1] = reinterpret_cast<const uint16_t*>(beta)[head];
-    } else {
-      reinterpret_cast<float*>(ab_head)[(n - 1) * 2 + 0] = reinterpret_cast<const float*>(alpha)[head];
-      reinterpret_cast<float*>(ab_head)[(n - 1) * 2 + 1] = reinterpret_cast<const float*>(beta)[head];
-    }
-  }
-  // earlier buffered tokens
-  for (int idx = tid; idx < (n - 1) * (int)row_elems; idx += kThreads) {
-    const int s = idx / (int)row_elems, e = idx - s * (int)row_elems;
-    const float x = load_io(kv_head, (size_t)s * row_elems + e, io);
-    if (e < d_k) Ks[s][e] = x; else Vs[s][e - d_k] = x;
-  }
-  for (int s = tid; s < n - 1; s += kThreads) {
-    al[s] = load_io(ab_head, (size_t)s * 2 + 0, io);
-    be[s] = load_io(ab_head, (size_t)s * 2 + 1, io);
-  }
-  // scales of the stored state
+  const int P = p.P;
   const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
-  const uint16_t* rsc = reinterpret_cast<const uint16_t*>(rec + code_bytes(d_k, d_v, bits));
-  for (int g = tid; g < p.n_groups; g += kThreads) sc[g] = __half2float(__ushort_as_half(rsc[g]));
-  __syncthreads();
 
-  // dot products: gram[t][s] = k_t.k_s (s < t), kq[s] = k_s.q
+  // 1. start streaming the first row blocks of codes
+  RowBlock<D, BITS> rbuf[PF];
+#pragma unroll
+  for (int r = 0; r < PF; ++r) rbuf[r].load(rec, r, g, t);
+
+  // 2. this token's inputs and the head's scales (lane holds elements EPL*lane..)
+  const size_t e0 = (size_t)head * D + (size_t)EPL * lane;
+  Raw<EPL, BF16> k_raw, v_raw;
+  k_raw.load(k, e0);
+  v_raw.load(v, e0);
+  float qf[EPL], kf[EPL], vf[EPL], sc[EPL];
+  load_f<EPL, BF16>(q, e0, qf);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    kf[e] = k_raw.get(e);
+    vf[e] = v_raw.get(e);
+  }
+  const float a_n = load_io(alpha, head, BF16 ? PACE_IO_BF16 : PACE_IO_F32);
+  const float b_n = load_io(beta, head, BF16 ? PACE_IO_BF16 : PACE_IO_F32);
   {
-    const int lane = tid & 31, warp = tid >> 5;
-    const int npairs = n * (n - 1) / 2;
-    for (int d = warp; d < npairs + n; d += kThreads / 32) {
-      int t, s;
-      const float* a;
-      const float* c;
-      if (d < npairs) {
-        t = 1;
-        while (t * (t + 1) / 2 <= d) ++t;
-        s = d - t * (t - 1) / 2;
-        a = Ks[t];
-        c = Ks[s];
+    Raw<EPL, true> s_raw;   // fp16 scales share the bf16 byte layout
+    s_raw.load(rec + code_bytes(D, D, BITS), (size_t)EPL * lane);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const uint32_t x = s_raw.w[e >> 1];
+      sc[e] = __half2float(__ushort_as_half((unsigned short)((e & 1) ? (x >> 16) : (x & 0xffff))));
+    }
+  }
+
+  // 3. dot products with the buffered keys: k_n.k_s and q.k_s
+  const size_t row_elems = 2 * (size_t)D;
+  const uint8_t* kv_head = p.kv + (size_t)head * P * row_elems * ESZ;
+  float part[2 * PMAX];
+#pragma unroll
+  for (int i = 0; i < 2 * PMAX; ++i) part[i] = 0.f;
+#pragma unroll
+  for (int s = 0; s < PMAX; ++s) {
+    if (s < n - 1) {
+      float ks[EPL];
+      load_f<EPL, BF16>(kv_head, s * row_elems + (size_t)EPL * lane, ks);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        part[s] = fmaf(kf[e], ks[e], part[s]);
+        part[PMAX + s] = fmaf(qf[e], ks[e], part[PMAX + s]);
+      }
+    } else if (s == n - 1) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) part[PMAX + s] = fmaf(qf[e], kf[e], part[PMAX + s]);
+    }
+  }
+  const float tot = transpose_reduce<2 * PMAX>(part, lane);
+  // lane s < PMAX: gk = k_n . k_s ; lane PMAX + s: q . k_s
+
+  // 4. per-token decays / gates, lane s = token s (0-based); lanes >= n neutral
+  float al = 1.f, be = 0.f;
+  const uint8_t* ab_head = p.ab + (size_t)head * p.ab_stride;
+  if (lane < n - 1) {
+    Raw<2, BF16> ab;
+    ab.load(ab_head, (size_t)lane * 2);
+    al = ab.get(0);
+    be = ab.get(1);
+  } else if (lane == n - 1) {
+    al = a_n;
+    be = b_n;
+  }
+  float gcum = al;                                     // gamma through token s
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float x = __shfl_up_sync(FULL, gcum, off);
+    if (lane >= off) gcum *= x;
+  }
+  float suf = __shfl_down_sync(FULL, al, 1);           // prod_{r > s} alpha_r
+  if (lane == 31) suf = 1.f;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float x = __shfl_down_sync(FULL, suf, off);
+    if (lane + off < 32) suf *= x;
+  }
+  const float gamma_n = __shfl_sync(FULL, gcum, n - 1);
+  const float w_s = suf * __shfl_sync(FULL, tot, (lane + PMAX) & 31);
+
+  // 5. column s of A: A[t][s] = beta_t gamma_{t/s} G[t][s], t > s
+  const float* gram_head = reinterpret_cast<const float*>(p.gram + (size_t)head * p.gram_stride);
+  float acol[PMAX];
+  float run = 1.f;
+#pragma unroll
+  for (int tt = 0; tt < PMAX; ++tt) {
+    const float at = __shfl_sync(FULL, al, tt);
+    const float bt = __shfl_sync(FULL, be, tt);
+    float G = 0.f;
+    if (tt > lane) {
+      run *= at;
+      if (tt < n - 1) G = gram_head[tt * P + lane];
+      else if (tt == n - 1) G = tot;
+    }
+    acol[tt] = (tt > lane && tt < n) ? bt * run * G : 0.f;
+  }
+  // 6. backward substitution (I + A^T) y = w, lane-parallel over s
+  float acc = w_s;
+#pragma unroll
+  for (int tt = PMAX - 1; tt >= 0; --tt) {
+    if (tt < n) {
+      const float yt = __shfl_sync(FULL, acc, tt);
+      if (lane < tt) acc = fmaf(-acol[tt], yt, acc);
+    }
+  }
+  const float z = be * acc;              // z_s (0 on lanes >= n)
+  const float zk = z * gcum;             // z_s gamma_s
+
+  // 7. q^ and the buffered-value term, lane-local over its EPL elements
+  float qh[EPL], vt[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    qh[e] = gamma_n * qf[e];
+    vt[e] = 0.f;
+  }
+#pragma unroll
+  for (int s = 0; s < PMAX; ++s) {
+    if (s < n) {
+      const float zks = __shfl_sync(FULL, zk, s);
+      const float zs = __shfl_sync(FULL, z, s);
+      float ks[EPL], vs[EPL];
+      if (s < n - 1) {
+        load_f<EPL, BF16>(kv_head, s * row_elems + (size_t)EPL * lane, ks);
+        load_f<EPL, BF16>(kv_head, s * row_elems + D + (size_t)EPL * lane, vs);
       } else {
-        t = -1;
-        s = d - npairs;
-        a = Ks[s];
-        c = qs;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) { ks[e] = kf[e]; vs[e] = vf[e]; }
       }
-      float acc = 0.f;
-      for (int j = lane; j < d_k; j += 32) acc = fmaf(a[j], c[j], acc);
-      for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) {
-        if (t >= 0) gram[t][s] = acc; else kq[s] = acc;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        qh[e] = fmaf(-zks, ks[e], qh[e]);
+        vt[e] = fmaf(zs, vs[e], vt[e]);
       }
     }
   }
-  __syncthreads();
 
-  // small n x n solve: y = (I + A)^{-T} w by backward substitution; z = beta * y
-  if (tid == 0) {
-    float y[PACE_MAX_PERIOD];
-    float gam[PACE_MAX_PERIOD + 1];
-    gam[0] = 1.f;
-    for (int t = 1; t <= n; ++t) gam[t] = gam[t - 1] * al[t - 1];       // gamma_t
-    for (int s = n; s >= 1; --s) {
-      float g_ns = 1.f;                                                   // gamma_{n/s}
-      for (int r = s + 1; r <= n; ++r) g_ns *= al[r - 1];
-      float acc = g_ns * kq[s - 1];
-      float g_ts = 1.f;                                                   // gamma_{t/s}
-      for (int t = s + 1; t <= n; ++t) {
-        g_ts *= al[t - 1];
-        const float a_ts = be[t - 1] * g_ts * gram[t - 1][s - 1];
-        acc -= a_ts * y[t - 1];
-      }
-      y[s - 1] = acc;
+  // 8. right-hand side b = q^ (times the column scales), normalised and split hi + lo
+  const bool col = p.axis == PACE_SCALE_COL;
+  float bv[EPL];
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    bv[e] = col ? qh[e] * sc[e] : qh[e];
+    m = fmaxf(m, fabsf(bv[e]));
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+  int ex = 0;
+  if (m > 0.f && m < INFINITY) ex = max(-100, min(100, 14 - ilogbf(m)));
+  const float up = ldexpf(1.f, ex), down = ldexpf(1.f, -ex);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const float x = bv[e] * up;
+    const __half hi = __float2half_rn(x);
+    const __half lo = __float2half_rn(x - __half2float(hi));
+    int tg, s, pos;
+    kslot_of<D, BITS>(EPL * lane + e, tg, s, pos);
+    scr.bfrag[0][tg][s][pos] = hi;
+    scr.bfrag[1][tg][s][pos] = lo;
+  }
+  __syncwarp();
+  uint32_t bfr[KS][2];
+  {
+    const int arr = g < 2 ? g : 2;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&scr.bfrag[arr][t][0][0]);
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+      bfr[s][0] = src[2 * s];
+      bfr[s][1] = src[2 * s + 1];
     }
-    for (int s = 1; s <= n; ++s) {
-      const float z = be[s - 1] * y[s - 1];
-      zv[s - 1] = z;
-      zk[s - 1] = z * gam[s];
+  }
+
+  // 9. y = S~0 (codes) x b on the tensor cores, 16 rows at a time
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    RowBlock<D, BITS> cur = rbuf[r % PF];
+    if (r + PF < RB) rbuf[r % PF].load(rec, r + PF, g, t);
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+      uint32_t a[4];
+      a_frag<D, BITS>(cur, s, a);
+      mma16816(d, a, bfr[s][0], bfr[s][1]);
     }
-    gamma_n = gam[n];
+    if (t == 0) {
+      scr.y[16 * r + g] = (d[0] + d[1]) * down;
+      scr.y[16 * r + g + 8] = (d[2] + d[3]) * down;
+    }
   }
-  __syncthreads();
+  __syncwarp();
 
-  // q^ = gamma_n q - sum_s z_s gamma_s k_s  (COL: folded with the column scales)
-  for (int j = tid; j < d_k; j += kThreads) {
-    float acc = gamma_n * qs[j];
-    for (int s = 0; s < n; ++s) acc = fmaf(-zk[s], Ks[s][j], acc);
-    qhat[j] = p.axis == PACE_SCALE_COL ? acc * sc[j] : acc;
+  // 10. o = (row scale) * y + sum_s z_s v_s
+  {
+    float out[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const float yv = scr.y[EPL * lane + e];
+      out[e] = (col ? yv : yv * sc[e]) + vt[e];
+    }
+    float* op = o + (size_t)head * D + (size_t)EPL * lane;
+    if (EPL == 4) *reinterpret_cast<float4*>(op) = make_float4(out[0], out[1], out[2], out[3]);
+    else if (EPL == 2) *reinterpret_cast<float2*>(op) = make_float2(out[0], out[1]);
+    else op[0] = out[0];
   }
-  __syncthreads();
 
-  // o_i = (S~0 q^)_i + sum_s z_s v_s[i]
-  const int row_bytes = d_k * bits / 8;
-  for (int i = tid; i < d_v; i += kThreads) {
-    float acc = 0.f;
-    for (int j = 0; j < d_k; ++j) acc = fmaf((float)decode_code(rec, row_bytes, i, j, bits), qhat[j], acc);
-    if (p.axis == PACE_SCALE_ROW) acc *= sc[i];
-    for (int s = 0; s < n; ++s) acc = fmaf(zv[s], Vs[s][i], acc);
-    o[(size_t)head * d_v + i] = acc;
+  // 11. buffer the token: k, v, alpha, beta, its Gram row; then fill = n
+  uint8_t* row = const_cast<uint8_t*>(kv_head) + (size_t)(n - 1) * row_elems * ESZ;
+  k_raw.store(row, (size_t)EPL * lane);
+  v_raw.store(row, D + (size_t)EPL * lane);
+  if (lane == 0) {
+    Raw<1, BF16> ra, rb2;
+    ra.load(alpha, head);
+    rb2.load(beta, head);
+    uint8_t* abp = const_cast<uint8_t*>(ab_head) + (size_t)(n - 1) * 2 * ESZ;
+    ra.store(abp, 0);
+    rb2.store(abp, 1);
   }
-  if (tid == 0) p.fill[head] = n;
+  if (lane < n - 1) const_cast<float*>(gram_head)[(n - 1) * P + lane] = tot;
+  __syncwarp();
+  if (lane == 0) p.fill[head] = n;
+}
+
+template <int D, bool BF16, int PMAX>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_step_kernel(PoolDev p, const void* __restrict__ q, const void* __restrict__ k,
+                       const void* __restrict__ v, const void* __restrict__ alpha,
+                       const void* __restrict__ beta, float* __restrict__ o) {
+  __shared__ WarpScratch<D> scratch[kWarpsPerBlock];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  WarpScratch<D>& scr = scratch[wib];
+  {
+    __half* z = &scr.bfrag[2][0][0][0];
+    for (int i = lane; i < 4 * (D / 16) * 4; i += 32) z[i] = __ushort_as_half((unsigned short)0);
+  }
+  __syncwarp();
+  const int n_heads = p.B * p.H;
+  const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
+  const int n_warps = gridDim.x * kWarpsPerBlock;
+  for (int head = warp0; head < n_heads; head += n_warps) {
+    int nprev = 0;
+    if (lane == 0) nprev = p.fill[head];
+    nprev = __shfl_sync(FULL, nprev, 0);
+    if (nprev < 0 || nprev >= p.P) {
+      if (lane == 0) atomicOr(p.flags, PACE_FLAG_BUFFER_FULL);
+      for (int i = lane; i < D; i += 32) o[(size_t)head * D + i] = __int_as_float(0x7fc00000);
+      continue;
+    }
+    const int n = nprev + 1;
+    if (p.bits[head % p.H] == 4)
+      decode_head<D, BF16, PMAX, 4>(p, head, n, q, k, v, alpha, beta, o, scr, lane);
+    else
+      decode_head<D, BF16, PMAX, 8>(p, head, n, q, k, v, alpha, beta, o, scr, lane);
+  }
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+template <int D, bool BF16, int PMAX>
+cudaError_t launch_t(const PoolDev& p, const void* q, const void* k, const void* v,
+                     const void* alpha, const void* beta, float* o, cudaStream_t st) {
+  const long heads = (long)p.B * p.H;
+  long blocks = (heads + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const long cap = 2L * sm_count();
+  if (blocks > cap) blocks = cap;
+  decode_step_kernel<D, BF16, PMAX><<<(unsigned)blocks, kThreads, 0, st>>>(p, q, k, v, alpha, beta, o);
+  return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t launch_p(const PoolDev& p, const void* q, const void* k, const void* v,
+                     const void* alpha, const void* beta, float* o, cudaStream_t st) {
+  if (p.P <= 4) return launch_t<D, BF16, 4>(p, q, k, v, alpha, beta, o, st);
+  if (p.P <= 8) return launch_t<D, BF16, 8>(p, q, k, v, alpha, beta, o, st);
+  return launch_t<D, BF16, 16>(p, q, k, v, alpha, beta, o, st);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_step(const PoolDev& p, const void* q, const void* k, const void* v,
                                const void* alpha, const void* beta, float* o, cudaStream_t st) {
-  decode_step_kernel<<<(unsigned)(p.B * p.H), kThreads, 0, st>>>(p, q, k, v, alpha, beta, o);
-  return cudaGetLastError();
+  const bool bf = p.io == PACE_IO_BF16;
+  switch (p.d_k) {
+    case 32: return bf ? launch_p<32, true>(p, q, k, v, alpha, beta, o, st)
+                       : launch_p<32, false>(p, q, k, v, alpha, beta, o, st);
+    case 64: return bf ? launch_p<64, true>(p, q, k, v, alpha, beta, o, st)
+                       : launch_p<64, false>(p, q, k, v, alpha, beta, o, st);
+    case 128: return bf ? launch_p<128, true>(p, q, k, v, alpha, beta, o, st)
+                        : launch_p<128, false>(p, q, k, v, alpha, beta, o, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace pace

@@ -22,7 +22,10 @@ struct PoolDev {
   uint64_t slot_stride;       // bytes per slot in the state region
   uint8_t* state;             // [B][slot_stride]
   uint8_t* kv;                // [B][H][P][d_k + d_v] io elements
-  uint8_t* ab;                // [B][H][P][2] io elements
+  uint8_t* ab;                // [B][H] blocks of ab_stride bytes: [P][2] io elements
+  uint8_t* gram;              // [B][H] blocks of gram_stride bytes: [P][P] fp32 k_t . k_s
+  uint32_t ab_stride;         // round_up(2 P io bytes, 16)
+  uint32_t gram_stride;       // round_up(4 P P, 16)
   int32_t* fill;              // [B][H]
   uint32_t* flags;            // status word
   uint32_t rec_off[PACE_MAX_HEADS];   // record offset of head h inside a slot
@@ -40,6 +43,14 @@ __host__ __device__ inline size_t record_bytes(int d_k, int d_v, int bits, int n
 }
 
 __host__ __device__ inline int io_size(int io) { return io == PACE_IO_BF16 ? 2 : 4; }
+
+__host__ __device__ inline uint32_t ab_stride_bytes(int P, int io) {
+  return (uint32_t)round_up((size_t)2 * P * io_size(io), 16);
+}
+
+__host__ __device__ inline uint32_t gram_stride_bytes(int P) {
+  return (uint32_t)round_up((size_t)4 * P * P, 16);
+}
 
 // Load element `idx` of an io-dtype array as fp32.
 __device__ __forceinline__ float load_io(const void* p, size_t idx, int io) {

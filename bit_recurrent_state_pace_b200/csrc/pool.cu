@@ -35,7 +35,7 @@ struct Layout {
   size_t slot_stride;
   size_t rec_off[PACE_MAX_HEADS];
   size_t rec_bytes[PACE_MAX_HEADS];
-  size_t state_bytes, kv_bytes, buffer_bytes, aux_bytes;
+  size_t state_bytes, kv_bytes, ab_bytes, buffer_bytes, aux_bytes;
   int n_groups;
 };
 
@@ -67,13 +67,15 @@ pace_status compute_layout(const pace_pool_desc* d, Layout* L) {
   L->slot_stride = round_up(off, 16);
   if (!mul_ok(L->slot_stride, (size_t)d->num_slots, &L->state_bytes)) return PACE_ERR_INVALID_ARG;
   const size_t esz = (size_t)pace::io_size(d->io_dtype);
-  size_t heads = 0, rows = 0, kv = 0, ab = 0;
+  size_t heads = 0, rows = 0, kv = 0, ab = 0, gram = 0;
   if (!mul_ok((size_t)d->num_slots, (size_t)d->num_heads, &heads)) return PACE_ERR_INVALID_ARG;
   if (!mul_ok(heads, (size_t)d->period, &rows)) return PACE_ERR_INVALID_ARG;
   if (!mul_ok(rows, (size_t)(d->d_k + d->d_v) * esz, &kv)) return PACE_ERR_INVALID_ARG;
-  if (!mul_ok(rows, 2 * esz, &ab)) return PACE_ERR_INVALID_ARG;
+  if (!mul_ok(heads, pace::ab_stride_bytes(d->period, d->io_dtype), &ab)) return PACE_ERR_INVALID_ARG;
+  if (!mul_ok(heads, pace::gram_stride_bytes(d->period), &gram)) return PACE_ERR_INVALID_ARG;
   L->kv_bytes = round_up(kv, 256);
-  L->buffer_bytes = L->kv_bytes + round_up(ab, 256);
+  L->ab_bytes = round_up(ab, 256);
+  L->buffer_bytes = L->kv_bytes + L->ab_bytes + round_up(gram, 256);
   L->aux_bytes = round_up(4 * heads, 256) + 256;
   if (heads > 0x7fffffffULL) return PACE_ERR_UNSUPPORTED;
   return PACE_OK;
@@ -139,6 +141,9 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
   dv.state = static_cast<uint8_t*>(d_state);
   dv.kv = static_cast<uint8_t*>(d_buffer);
   dv.ab = static_cast<uint8_t*>(d_buffer) + L.kv_bytes;
+  dv.gram = static_cast<uint8_t*>(d_buffer) + L.kv_bytes + L.ab_bytes;
+  dv.ab_stride = pace::ab_stride_bytes(desc->period, desc->io_dtype);
+  dv.gram_stride = pace::gram_stride_bytes(desc->period);
   dv.fill = static_cast<int32_t*>(d_aux);
   dv.flags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(d_aux) + L.aux_bytes - 256);
   for (int h = 0; h < desc->num_heads; ++h) {

@@ -86,9 +86,14 @@ typedef struct {
  * buffer : the token buffer ([P2] "Periodic Rounding"; [P4] flowchart "Small
  *          buffer, last few tokens"): region KV = [B][H][P][d_k + d_v]
  *          io_dtype elements (row = k then v of one buffered token), then at
- *          byte offset round_up(size(KV), 256) region AB = [B][H][P][2]
- *          io_dtype elements (alpha, beta).  q is not stored: no later step
- *          reads an old query.
+ *          byte offset round_up(size(KV), 256) region AB: [B][H] blocks of
+ *          round_up(2*P*io_size, 16) bytes, each [P][2] io_dtype elements
+ *          (alpha, beta); then at the next 256-byte boundary region G: [B][H]
+ *          blocks of round_up(4*P*P, 16) bytes, each [P][P] fp32 with
+ *          G[t][s] = k_t . k_s for s < t, the Gram entries of the buffered
+ *          keys, written by the decode step that buffers token t (so each step
+ *          computes only its own).  q is not stored: no later step reads an
+ *          old query.
  * aux    : fill counters int32 [B][H] (tokens in each head's buffer), then at
  *          byte offset round_up(4*B*H, 256) the uint32 status word.
  * All three regions must be 256-byte aligned.
