@@ -40,6 +40,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["pace", "reference"], default="pace")
     ap.add_argument("--workload", default="concurrency_stress")
     ap.add_argument("--period", type=int, default=None, help="override P")
+    ap.add_argument("--slots", type=int, default=None, help="override B (smaller profiling case)")
     ap.add_argument("--prefill", type=int, default=None, help="warm-up prefill tokens (default: workload's)")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
@@ -233,6 +234,8 @@ def run_pace(args, rank: int, world: int):
         w = w.replace(P=args.period)
     if args.prefill is not None:
         w = w.replace(warmup=args.prefill)
+    if args.slots is not None:
+        w = w.replace(B=args.slots)
     bits = pace_synth.head_bits(w, args.seed)
     BH, P = w.B * w.H, w.P
     stream = torch.cuda.current_stream()

@@ -25,6 +25,7 @@
 // warp shuffles; k.k dot products of earlier buffered tokens are cached in
 // the buffer's Gram region, so each step computes only the 2n-1 new ones.
 #include "frag.cuh"
+#include "tma.cuh"
 
 namespace pace {
 
@@ -312,10 +313,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int n_heads = p.B * p.H;
   const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
   const int n_warps = gridDim.x * kWarpsPerBlock;
+  constexpr int ESZ = BF16 ? 2 : 4;
+  int fill_next = 0;
+  if (lane == 0 && warp0 < n_heads) fill_next = p.fill[warp0];
   for (int head = warp0; head < n_heads; head += n_warps) {
-    int nprev = 0;
-    if (lane == 0) nprev = p.fill[head];
-    nprev = __shfl_sync(FULL, nprev, 0);
+    int nprev = __shfl_sync(FULL, fill_next, 0);
+    // start the next head of this warp on its way into L2: its record and
+    // inputs now, its buffered rows once its fill count is known
+    const int nh = head + n_warps;
+    if (lane == 0 && nh < n_heads) {
+      const int hh = nh % p.H;
+      prefetch_l2(p.state + (size_t)(nh / p.H) * p.slot_stride + p.rec_off[hh],
+                  (uint32_t)record_bytes(D, D, p.bits[hh], D));
+      prefetch_l2(reinterpret_cast<const uint8_t*>(q) + (size_t)nh * D * ESZ, D * ESZ);
+      prefetch_l2(reinterpret_cast<const uint8_t*>(k) + (size_t)nh * D * ESZ, D * ESZ);
+      prefetch_l2(reinterpret_cast<const uint8_t*>(v) + (size_t)nh * D * ESZ, D * ESZ);
+      fill_next = p.fill[nh];
+    }
     if (nprev < 0 || nprev >= p.P) {
       if (lane == 0) atomicOr(p.flags, PACE_FLAG_BUFFER_FULL);
       for (int i = lane; i < D; i += 32) o[(size_t)head * D + i] = __int_as_float(0x7fc00000);
@@ -326,6 +340,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       decode_head<D, BF16, PMAX, 4>(p, head, n, q, k, v, alpha, beta, o, scr, lane);
     else
       decode_head<D, BF16, PMAX, 8>(p, head, n, q, k, v, alpha, beta, o, scr, lane);
+    if (lane == 0 && nh < n_heads && fill_next > 0 && fill_next < p.P) {
+      prefetch_l2(p.kv + (size_t)nh * p.P * 2 * D * ESZ, (uint32_t)(fill_next * 2 * D * ESZ));
+      prefetch_l2(p.ab + (size_t)nh * p.ab_stride, p.ab_stride);
+      prefetch_l2(p.gram + (size_t)nh * p.gram_stride, p.gram_stride);
+    }
   }
 }
 
