@@ -37,7 +37,7 @@ constexpr unsigned FULL = 0xffffffffu;
 
 template <int D>
 struct alignas(16) WarpScratch {
-  __half bfrag[3][4][D / 16][4];   // [hi | lo | zero][lane group t][k-step][pos]
+  uint8_t dig[4][D];               // digits 0..2 of the right-hand side, row 3 = zeros
   float y[D];                      // S~0 q^ by row, before the row scale
 };
 
@@ -211,7 +211,8 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     }
   }
 
-  // 8. right-hand side b = q^ (times the column scales), normalised and split hi + lo
+  // 8. right-hand side b = q^ (times the column scales) as 22-bit fixed point,
+  //    split into three balanced base-256 digits: b 2^e = d0 + 256 d1 + 65536 d2
   const bool col = p.axis == PACE_SCALE_COL;
   float bv[EPL];
   float m = 0.f;
@@ -223,45 +224,108 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
 #pragma unroll
   for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
   int ex = 0;
-  if (m > 0.f && m < INFINITY) ex = max(-100, min(100, 14 - ilogbf(m)));
+  if (m > 0.f && m < INFINITY) ex = max(-120, min(120, 21 - ilogbf(m)));
   const float up = ldexpf(1.f, ex), down = ldexpf(1.f, -ex);
+  int dsum[3] = {0, 0, 0};
+  uint32_t dw[3] = {0u, 0u, 0u};    // digit bytes of this lane's EPL elements
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
-    const float x = bv[e] * up;
-    const __half hi = __float2half_rn(x);
-    const __half lo = __float2half_rn(x - __half2float(hi));
-    int tg, s, pos;
-    kslot_of<D, BITS>(EPL * lane + e, tg, s, pos);
-    scr.bfrag[0][tg][s][pos] = hi;
-    scr.bfrag[1][tg][s][pos] = lo;
+    const int Q = __float2int_rn(bv[e] * up);
+    const int d0 = (int)(int8_t)(Q & 0xff);
+    const int r1 = (Q - d0) >> 8;
+    const int d1 = (int)(int8_t)(r1 & 0xff);
+    const int d2 = (r1 - d1) >> 8;
+    dsum[0] += d0; dsum[1] += d1; dsum[2] += d2;
+    dw[0] |= (uint32_t)(d0 & 0xff) << (8 * e);
+    dw[1] |= (uint32_t)(d1 & 0xff) << (8 * e);
+    dw[2] |= (uint32_t)(d2 & 0xff) << (8 * e);
   }
-  __syncwarp();
-  uint32_t bfr[KS][2];
-  {
-    const int arr = g < 2 ? g : 2;
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(&scr.bfrag[arr][t][0][0]);
+  if (BITS == 8) {
+    // natural key-channel order
 #pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      bfr[s][0] = src[2 * s];
-      bfr[s][1] = src[2 * s + 1];
+    for (int d = 0; d < 3; ++d) {
+      uint8_t* dst = &scr.dig[d][EPL * lane];
+      if (EPL == 4) *reinterpret_cast<uint32_t*>(dst) = dw[d];
+      else if (EPL == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)dw[d];
+      else *dst = (uint8_t)dw[d];
+    }
+  } else {
+    // within each group of 8 key channels: even offsets first, then odd
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int j = EPL * lane + e, o = j & 7;
+      const int at = (j & ~7) + ((o & 1) ? 4 + (o >> 1) : (o >> 1));
+#pragma unroll
+      for (int d = 0; d < 3; ++d) scr.dig[d][at] = (uint8_t)(dw[d] >> (8 * e));
     }
   }
+  // INT4 codes enter the tensor cores as offset bytes c + 8: remove 8 sum(digits)
+  int corr[3] = {0, 0, 0};
+  if (BITS == 4) {
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+      int v2 = dsum[d];
+#pragma unroll
+      for (int off = 16; off; off >>= 1) v2 += __shfl_xor_sync(FULL, v2, off);
+      corr[d] = 8 * v2;
+    }
+  }
+  __syncwarp();
+  constexpr int NC = D / 32;           // k32 chunks
+  uint32_t bfr[NC][2];
+  {
+    const uint8_t* src = &scr.dig[g < 3 ? g : 3][0];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      if (BITS == 4) {
+        const int at = (D / 4) * t + 8 * c;
+        bfr[c][0] = *reinterpret_cast<const uint32_t*>(src + at);
+        bfr[c][1] = *reinterpret_cast<const uint32_t*>(src + at + 4);
+      } else {
+        const int m0 = 2 * c, m1 = 2 * c + 1;
+        const int j0 = m0 < NC ? (D / 8) * t + 4 * m0 : D / 2 + (D / 8) * t + 4 * (m0 - NC);
+        const int j1 = m1 < NC ? (D / 8) * t + 4 * m1 : D / 2 + (D / 8) * t + 4 * (m1 - NC);
+        bfr[c][0] = *reinterpret_cast<const uint32_t*>(src + j0);
+        bfr[c][1] = *reinterpret_cast<const uint32_t*>(src + j1);
+      }
+    }
+  }
+  const int cA = t == 0 ? corr[0] : corr[2];
+  const int cB = t == 0 ? corr[1] : 0;
 
-  // 9. y = S~0 (codes) x b on the tensor cores, 16 rows at a time
+  // 9. y = S~0 (codes) x b on the int8 tensor cores (exact int32), 16 rows at a time
 #pragma unroll
   for (int r = 0; r < RB; ++r) {
     RowBlock<D, BITS> cur = rbuf[r % PF];
     if (r + PF < RB) rbuf[r % PF].load(rec, r + PF, g, t);
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    int d[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int s = 0; s < KS; ++s) {
+    for (int c = 0; c < NC; ++c) {
       uint32_t a[4];
-      a_frag<D, BITS>(cur, s, a);
-      mma16816(d, a, bfr[s][0], bfr[s][1]);
+      if (BITS == 4) {
+        const uint32_t w0 = cur.w[0][c], w1 = cur.w[1][c];
+        a[0] = (w0 & 0x0F0F0F0Fu) ^ 0x08080808u;
+        a[1] = (w1 & 0x0F0F0F0Fu) ^ 0x08080808u;
+        a[2] = ((w0 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+        a[3] = ((w1 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+        mma_u8s8(d, a, bfr[c][0], bfr[c][1]);
+      } else {
+        a[0] = cur.w[0][2 * c];
+        a[1] = cur.w[1][2 * c];
+        a[2] = cur.w[0][2 * c + 1];
+        a[3] = cur.w[1][2 * c + 1];
+        mma_s8s8(d, a, bfr[c][0], bfr[c][1]);
+      }
     }
+    // columns 0, 1, 2 = digits: lane t = 0 holds d0, d1; lane t = 1 holds d2
+    const float wB = t == 0 ? 256.f : 0.f, wA = t == 0 ? 1.f : 65536.f;
+    float pg = wA * (float)(d[0] - cA) + wB * (float)(d[1] - cB);
+    float ph = wA * (float)(d[2] - cA) + wB * (float)(d[3] - cB);
+    pg += __shfl_down_sync(FULL, pg, 1);
+    ph += __shfl_down_sync(FULL, ph, 1);
     if (t == 0) {
-      scr.y[16 * r + g] = (d[0] + d[1]) * down;
-      scr.y[16 * r + g + 8] = (d[2] + d[3]) * down;
+      scr.y[16 * r + g] = pg * down;
+      scr.y[16 * r + g + 8] = ph * down;
     }
   }
   __syncwarp();
@@ -305,10 +369,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ WarpScratch<D> scratch[kWarpsPerBlock];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   WarpScratch<D>& scr = scratch[wib];
-  {
-    __half* z = &scr.bfrag[2][0][0][0];
-    for (int i = lane; i < 4 * (D / 16) * 4; i += 32) z[i] = __ushort_as_half((unsigned short)0);
-  }
+  for (int i = lane; i < D; i += 32) scr.dig[3][i] = 0;
   __syncwarp();
   const int n_heads = p.B * p.H;
   const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
