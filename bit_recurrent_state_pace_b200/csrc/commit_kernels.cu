@@ -19,15 +19,19 @@
 // over a persistent grid, the next head's record, buffered rows, gates and
 // Gram block brought into shared memory by 1-D TMA bulk copies while the
 // current head computes (double buffer, mbarrier completion, bounded waits).
-// Both contractions run on the tensor cores (mma.sync m16n8k16, f16
-// operands, fp32 accumulation):
-//   X:      A = codes (exact), B = K (times column scales) split hi + lo;
-//   update: A = U^ split hi + lo, B = K, accumulator initialised with
-//           gamma_P S~0 (the same fragments' codes times their scales),
-// so the fp32 period-end state of a 16 x D row block lives in registers.
-// Column absmax: per-lane pairs, a shuffle transpose over the 8 row lanes and
-// a shared-memory max over the warps; the new codes are rounded with the
-// f16 magic-number conversion (1032 + c, 1152 + c) and packed back in place.
+// Both contractions run on the f16 tensor cores (mma.sync m16n8k16, fp32
+// accumulation); the codes are exact in f16 and every fp32 operand is split
+// hi + lo after a power-of-two normalisation:
+//   X:      A = codes, B = the keys (times the column scales);
+//   update: A = U^, B = K, accumulator initialised with gamma_P S~0 from the
+//           same code fragments.
+// The update's output columns follow the code fragments' key channels, so
+// the initialisation, the column absmax and the re-encode stay lane-local.
+// Column absmax: per-lane row pairs, a shuffle transpose over the 8 row lanes
+// and a shared-memory max over the warps; the new codes are rounded with the
+// f16 magic-number conversion (1032 + c, 1152 + c) and packed in place.
+#include <type_traits>
+
 #include "encode.cuh"
 #include "frag.cuh"
 #include "tma.cuh"
@@ -37,6 +41,11 @@ namespace pace {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
+
+// floor(log2(m)) for a positive normal float, from its exponent bits
+__device__ __forceinline__ int exp2_floor(float m) { return (int)((__float_as_uint(m) >> 23) & 0xffu) - 127; }
+// 2^e for e in [-126, 127], exact
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
 
 __device__ __forceinline__ float max_nan(float a, float b) {
   float r;
@@ -51,40 +60,37 @@ struct Cfg {
   static constexpr int KS = D / 16;                 // k16 steps over key channels
   static constexpr int NT = D / 8;                  // n8 output tiles per row block
   static constexpr int NTX = (2 * PMAX + 7) / 8;    // X tiles: P vectors x (hi, lo)
-  static constexpr int NSEG = BF16 ? 2 : 3;         // update K segments
+  static constexpr int NSEG = BF16 ? 2 : 3;         // update K segments: hi | lo (| hi x k_lo)
   static constexpr int KU = (NSEG * PMAX + 15) / 16;  // update k16 steps
-  static constexpr int NU = PMAX >= 16 ? 4 : 2;     // distinct U^ rows a lane needs
+  static constexpr int NU = PMAX >= 16 ? 4 : 2;     // distinct U^ rows a lane feeds
   static constexpr int ESZ = BF16 ? 2 : 4;
   static constexpr int REC = (D * D + 2 * D + 15) / 16 * 16;   // largest record (INT8)
   static constexpr int KVB = PMAX * 2 * D * ESZ;
   static constexpr int ABB = (2 * PMAX * ESZ + 15) / 16 * 16;
-  static constexpr int GRB = (4 * PMAX * PMAX + 15) / 16 * 16;
+  static constexpr int GRB = (4 * PMAX * (PMAX + 1) + 15) / 16 * 16;
   static constexpr int SLOT = REC + KVB + ABB + GRB;
+};
+
+template <int D>
+struct alignas(16) WarpTab {
+  float4 f[D / 16][4];            // [ks][t]: up * gamma_P * s_j at the lane's 4 fragment channels
+  float4 q[D / 16][4];            // [ks][t]: this warp's quantisation factors, same order
 };
 
 template <int D, bool BF16, int PMAX>
 struct alignas(16) Smem {
   using C = Cfg<D, BF16, PMAX>;
-  uint8_t slot[2][C::SLOT];                     // staged record | kv rows | gates | Gram
-  uint32_t bx[C::NTX][C::KS][8][4][2];          // X B fragments [tile][ks][g][t][b0,b1]
-  __half bk[D][C::KU * 16 + 2];                 // update B: [key channel][slot] (+2: banks)
-  float F[C::KS][4][4];                         // COL: gamma_P s_j, [ks][t][pos]
-  float qfr[C::KS][4][4];                       // COL: new 1/s16, [ks][t][pos]
-  float sfr[C::KS][4][4];                       // COL: new s16 as float, [ks][t][pos]
-  float rowv[D];                                // ROW: gamma_P s_i
-  float rowq[D], rows[D];                       // ROW: new 1/s16 and s16 per row
-  float sc[D];                                  // old scales as float
-  float vf[PMAX][D];                            // buffered values, fp32
-  float A[PMAX][PMAX];
-  float W[PMAX][PMAX];
-  float gam[PMAX];
-  float xinv[PMAX];
+  uint8_t slot[2][C::SLOT];                       // staged record | kv rows | gates | Gram
+  uint2 bx[C::NTX][C::KS][8][4];                  // X B fragments [tile][ks][g][t]
+  uint2 bkf[C::NT][C::KU][8][4];                  // update B fragments [tile][u][g][t]
+  float sc[D];                                    // old scales (float)
+  float qf[D], sfv[D];                            // new 1/s16 and s16 (column or row)
   float colmax[C::RB][D];
+  WarpTab<D> wt[C::RB];
   uint64_t bar[2];
-  float gP;
+  float xinv;
   int next_head;
   int slow;
-  int abort_;
 };
 
 __device__ __forceinline__ int find_full(const PoolDev& p, int from, int step, int n_heads) {
@@ -142,12 +148,11 @@ __device__ __forceinline__ void load_rows_smem(RowBlock<D, BITS>& rb, const uint
   }
 }
 
-// f16x2 "magic" values of two codes: the mantissa holds code + 8 (INT4) or
-// code + 128 (INT8) on top of 1024.
 template <int BITS>
 __device__ __forceinline__ uint32_t magic_fast(float a, float b, float qa, float qb) {
   const float M = BITS == 4 ? 1032.f : 1152.f;
-  return h2u(__floats2half2_rn(fmaf(a, qa, M), fmaf(b, qb, M)));
+  const float2 r = __ffma2_rn(make_float2(a, b), make_float2(qa, qb), make_float2(M, M));
+  return h2u(__floats2half2_rn(r.x, r.y));
 }
 
 template <int BITS>
@@ -158,24 +163,15 @@ __device__ __forceinline__ uint32_t magic_exact(float a, float b, float sa, floa
   return (0x6400u | ca) | ((0x6400u | cb) << 16);
 }
 
-// Four f16x2 magic values of code pairs (8m+0,8m+4), (8m+1,8m+5), (8m+2,8m+6),
-// (8m+3,8m+7) -> one word of eight 4-bit two's complement codes.
-__device__ __forceinline__ uint32_t pack_int4(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3) {
-  // low nibble of each f16 half = code + 8; flipping bit 3 gives the 4-bit two's complement
-  const uint32_t m0 = (p0 & 0x000F000Fu) ^ 0x00080008u, m1 = (p1 & 0x000F000Fu) ^ 0x00080008u;
-  const uint32_t m2 = (p2 & 0x000F000Fu) ^ 0x00080008u, m3 = (p3 & 0x000F000Fu) ^ 0x00080008u;
-  return m0 | (m1 << 4) | (m2 << 8) | (m3 << 12);
-}
-
-// Two f16x2 magic values (codes j, j+1) and (j+2, j+3) -> four INT8 codes.
-__device__ __forceinline__ uint32_t pack_int8(uint32_t lo, uint32_t hi) {
-  return prmt(lo, hi, 0x6420u) ^ 0x80808080u;
+__device__ __forceinline__ float pick4(const float4& f, int i) {
+  return i == 0 ? f.x : i == 1 ? f.y : i == 2 ? f.z : f.w;
 }
 
 template <int D, bool BF16, int PMAX, int BITS>
 __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot) {
   using C = Cfg<D, BF16, PMAX>;
   constexpr int KS = C::KS, NT = C::NT, NTX = C::NTX, KU = C::KU, NU = C::NU;
+  constexpr int ROWB = D * BITS / 8;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
   const int P = p.P, h = head % p.H, b = head / p.H;
   const bool col = p.axis == PACE_SCALE_COL;
@@ -189,143 +185,127 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   const uint16_t* s_sc = reinterpret_cast<const uint16_t*>(s_rec + code_bytes(D, D, BITS));
 
   // ---- phase 1: per-head operands ------------------------------------------
-  float gP = 1.f;
-  for (int s = 0; s < P; ++s) gP *= io_at(s_ab, 2 * s, BF16);
-  for (int j = tid; j < D; j += C::THREADS) {
-    const float s = __half2float(__ushort_as_half(s_sc[j]));
-    sm.sc[j] = s;
-    sm.rowv[j] = gP * s;
-  }
-  for (int idx = tid; idx < 4 * KS * 4; idx += C::THREADS) {
-    const int tt = idx / (KS * 4), ks = (idx / 4) % KS, pos = idx & 3;
-    const int j = jof<D, BITS>(tt, ks, pos);
-    sm.F[ks][tt][pos] = gP * __half2float(__ushort_as_half(s_sc[j]));
-  }
-  for (int idx = tid; idx < P * D; idx += C::THREADS) {
-    const int s = idx / D, i = idx - s * D;
-    sm.vf[s][i] = io_at(s_kv, s * 2 * D + D + i, BF16);
-  }
-  for (int idx = tid; idx < D * P; idx += C::THREADS) {      // update B: K (hi, hi | lo)
-    const int j = idx / P, s = idx - (idx / P) * P;
-    const float kv = io_at(s_kv, s * 2 * D + j, BF16);
-    const __half hi = __float2half_rn(kv);
-    sm.bk[j][s] = hi;
-    sm.bk[j][PMAX + s] = hi;
-    if (C::NSEG == 3) sm.bk[j][2 * PMAX + s] = __float2half_rn(kv - __half2float(hi));
-  }
-  if (w == 0) {
-    // gates, decay products, A, T = (I + A)^{-1} and W, lane s = token s
-    const float al = lane < P ? io_at(s_ab, 2 * lane, BF16) : 1.f;
-    const float be = lane < P ? io_at(s_ab, 2 * lane + 1, BF16) : 0.f;
-    float gcum = al;
+  // W[s][s'] (P x P) and gamma_s (P) were left in the Gram block by the decode
+  // step that buffered the P-th token.
+  const float* W = s_gr;
+  const float* gam = s_gr + P * P;
+  const float gP = gam[P - 1];
+  for (int j = tid; j < D; j += C::THREADS) sm.sc[j] = __half2float(__ushort_as_half(s_sc[j]));
+  {
+    // one power-of-two normalisation of the X operand for the whole head, from
+    // the largest column scale (COL) and the largest |k| of the period
+    float smax = 0.f, kmax = 0.f;
+    for (int j = lane; j < D; j += 32) smax = fmaxf(smax, __half2float(__ushort_as_half(s_sc[j])));
+    constexpr int EPW = 16 / C::ESZ;                       // elements per 16-byte load
+    for (int i = lane; i < P * D / EPW; i += 32) {
+      const int s2 = i / (D / EPW), jv = i - s2 * (D / EPW);
+      const uint4 v4 = *reinterpret_cast<const uint4*>(s_kv + (size_t)(s2 * 2 * D + jv * EPW) * C::ESZ);
+      const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float x = __shfl_up_sync(FULL, gcum, off);
-      if (lane >= off) gcum *= x;
-    }
-    float suf = __shfl_down_sync(FULL, al, 1);
-    if (lane == 31) suf = 1.f;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float x = __shfl_down_sync(FULL, suf, off);
-      if (lane + off < 32) suf *= x;
-    }
-    float run = 1.f;
-#pragma unroll
-    for (int tt = 0; tt < PMAX; ++tt) {
-      const float at = __shfl_sync(FULL, al, tt), bt = __shfl_sync(FULL, be, tt);
-      float a = 0.f;
-      if (tt > lane) {
-        run *= at;
-        if (tt < P && lane < P) a = bt * run * s_gr[tt * P + lane];
-      }
-      if (lane < PMAX) sm.A[tt][lane] = a;
-    }
-    __syncwarp();
-    float Tc[PMAX];
-#pragma unroll
-    for (int tt = 0; tt < PMAX; ++tt) {
-      float acc = 0.f;
-#pragma unroll
-      for (int r = 0; r < tt; ++r)
-        if (r >= lane) acc = fmaf(sm.A[tt][r], Tc[r], acc);
-      Tc[tt] = tt == lane ? 1.f : (tt > lane ? -acc : 0.f);
-    }
-#pragma unroll
-    for (int tt = 0; tt < PMAX; ++tt) {
-      const float sf_t = __shfl_sync(FULL, suf, tt);
-      if (lane < PMAX) sm.W[tt][lane] = (tt < P && lane < P) ? sf_t * Tc[tt] * be : 0.f;
-    }
-    if (lane < PMAX) sm.gam[lane] = gcum;
-  } else {
-    // X operand: vector s (scaled by column scales in COL mode), normalised, hi/lo
-    for (int s = w - 1; s < P; s += C::RB - 1) {
-      constexpr int E = D / 32;
-      float val[E];
-      float m = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int j = lane + 32 * e;
-        const float kv = io_at(s_kv, s * 2 * D + j, BF16);
-        val[e] = col ? kv * __half2float(__ushort_as_half(s_sc[j])) : kv;
-        m = fmaxf(m, fabsf(val[e]));
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
-      int ex = 0;
-      if (m > 0.f && m < INFINITY) ex = max(-60, min(60, 14 - ilogbf(m)));
-      const float up = ldexpf(1.f, ex);
-      if (lane == 0) sm.xinv[s] = ldexpf(1.f, -ex);
-      __half* bxh = reinterpret_cast<__half*>(&sm.bx[0][0][0][0][0]);
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int j = lane + 32 * e;
-        const float x = val[e] * up;
-        const __half hi = __float2half_rn(x);
-        const __half lo = __float2half_rn(x - __half2float(hi));
-        int tt, ks, pos;
-        kslot_of<D, BITS>(j, tt, ks, pos);
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const int c = 2 * s + part, tile = c >> 3, gc = c & 7;
-          const size_t at = ((((size_t)tile * KS + ks) * 8 + gc) * 4 + tt) * 4 + pos;
-          bxh[at] = part ? lo : hi;
+      for (int e = 0; e < 4; ++e) {
+        if (BF16) {
+          kmax = fmaxf(kmax, __uint_as_float((wv[e] << 16) & 0x7fffffffu));
+          kmax = fmaxf(kmax, __uint_as_float(wv[e] & 0x7fff0000u));
+        } else {
+          kmax = fmaxf(kmax, __uint_as_float(wv[e] & 0x7fffffffu));
         }
       }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, off));
+      kmax = fmaxf(kmax, __shfl_xor_sync(FULL, kmax, off));
+    }
+    const float bmax = col ? smax * kmax : kmax;
+    int exx = 0;
+    if (bmax >= 1.17549435e-38f && bmax < INFINITY) exx = max(-120, min(120, 14 - exp2_floor(bmax)));
+    const float upx = pow2i(exx);
+    if (tid == 0) sm.xinv = pow2i(-exx);
+    // X operand: element (s, j) -> hi / lo f16 at its fragment position in
+    // columns 2s / 2s+1 (8 columns per tile)
+    __half* bxh = reinterpret_cast<__half*>(&sm.bx[0][0][0][0]);
+    for (int idx = tid; idx < P * D; idx += C::THREADS) {
+      const int s = idx / D, j = idx - (idx / D) * D;
+      const float kv = io_at(s_kv, s * 2 * D + j, BF16);
+      const float x = (col ? kv * __half2float(__ushort_as_half(s_sc[j])) : kv) * upx;
+      const __half hi = __float2half_rn(x);
+      const __half lo = __float2half_rn(x - __half2float(hi));
+      int tt, ks, pos;
+      kslot_of<D, BITS>(j, tt, ks, pos);
+      const int c0 = 2 * s, tile = c0 >> 3, gc = c0 & 7;
+      const size_t at = ((((size_t)tile * KS + ks) * 8 + gc) * 4 + tt) * 4 + pos;
+      bxh[at] = hi;
+      bxh[at + 16] = lo;                         // column gc + 1 of the same tile
+    }
+    // update B: column n = g of tile 2ks + hs is key channel jof(g>>1, ks, 2hs + (g&1));
+    // k-step u, lane group t holds slots 16u + 2t + {0, 1} (b0) and + {8, 9} (b1);
+    // slot sigma is token sigma % PMAX of segment sigma / PMAX (K, K, K_lo)
+    for (int cix = tid; cix < NT * 8; cix += C::THREADS) {
+      const int tau = cix >> 3, gg = cix & 7;
+      const int j = jof<D, BITS>(gg >> 1, tau >> 1, 2 * (tau & 1) + (gg & 1));
+      __half kh[PMAX], kl[PMAX];
+#pragma unroll
+      for (int s2 = 0; s2 < PMAX; ++s2) {
+        const float kv = s2 < P ? io_at(s_kv, s2 * 2 * D + j, BF16) : 0.f;
+        kh[s2] = __float2half_rn(kv);
+        kl[s2] = C::NSEG == 3 ? __float2half_rn(kv - __half2float(kh[s2])) : kh[s2];
+      }
+#pragma unroll
+      for (int u = 0; u < KU; ++u)
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          uint32_t wv[2];
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            __half hv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int sigma = 16 * u + 2 * tt + e + 8 * q2;
+              const int seg = sigma / PMAX, s2 = sigma % PMAX;
+              hv[e] = seg >= C::NSEG ? __ushort_as_half((unsigned short)0) : (seg == 2 ? kl[s2] : kh[s2]);
+            }
+            wv[q2] = h2u(__halves2half2(hv[0], hv[1]));
+          }
+          sm.bkf[tau][u][gg][tt] = make_uint2(wv[0], wv[1]);
+        }
     }
   }
   __syncthreads();
 
   // ---- phase 2: this warp's 16 rows ------------------------------------------
   const int i0 = 16 * w + g, i1 = i0 + 8;
-  RowBlock<D, BITS> rbk;
-  load_rows_smem<D, BITS>(rbk, s_rec, w, g, t);
   uint32_t Af[KS][4];
+  {
+    RowBlock<D, BITS> rbk;
+    load_rows_smem<D, BITS>(rbk, s_rec, w, g, t);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) a_frag<D, BITS>(rbk, ks, Af[ks]);
+  }
+  // X = S~0 K^T: column 2s = hi, 2s+1 = lo of vector s
   float xacc[NTX][4];
 #pragma unroll
   for (int x = 0; x < NTX; ++x) xacc[x][0] = xacc[x][1] = xacc[x][2] = xacc[x][3] = 0.f;
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    a_frag<D, BITS>(rbk, ks, Af[ks]);
+  for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
     for (int x = 0; x < NTX; ++x) {
-      const uint2 bb = *reinterpret_cast<const uint2*>(&sm.bx[x][ks][g][t][0]);
+      const uint2 bb = sm.bx[x][ks][g][t];
       mma16816(xacc[x], Af[ks], bb.x, bb.y);
     }
-  }
   // r_s = v_s - gamma_s x_s for this lane's vectors s = 4x + t, then all-gather in the quad
   float r[PMAX][2];
   {
     float ro[NTX][2];
-    const float s0 = col ? 1.f : sm.sc[i0], s1 = col ? 1.f : sm.sc[i1];
+    const float xinv = sm.xinv;
+    const float s0 = (col ? 1.f : sm.sc[i0]) * xinv, s1 = (col ? 1.f : sm.sc[i1]) * xinv;
 #pragma unroll
     for (int x = 0; x < NTX; ++x) {
       const int s = 4 * x + t;
       ro[x][0] = ro[x][1] = 0.f;
       if (s < P) {
-        const float xi = sm.xinv[s], gs = sm.gam[s];
-        ro[x][0] = sm.vf[s][i0] - gs * ((xacc[x][0] + xacc[x][1]) * xi * s0);
-        ro[x][1] = sm.vf[s][i1] - gs * ((xacc[x][2] + xacc[x][3]) * xi * s1);
+        const float gs = gam[s];
+        ro[x][0] = io_at(s_kv, s * 2 * D + D + i0, BF16) - gs * ((xacc[x][0] + xacc[x][1]) * s0);
+        ro[x][1] = io_at(s_kv, s * 2 * D + D + i1, BF16) - gs * ((xacc[x][2] + xacc[x][3]) * s1);
       }
     }
 #pragma unroll
@@ -350,7 +330,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int sp = 0; sp < PMAX; ++sp) {
-      const float wv = sm.W[s][sp];
+      const float wv = (s < P && sp < P) ? W[s * P + sp] : 0.f;
       a0 = fmaf(wv, r[sp][0], a0);
       a1 = fmaf(wv, r[sp][1], a1);
     }
@@ -361,8 +341,8 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 #pragma unroll
   for (int off = 16; off; off >>= 1) um = fmaxf(um, __shfl_xor_sync(FULL, um, off));
   int ex = 0;
-  if (um > 0.f && um < INFINITY) ex = max(-60, min(60, 14 - ilogbf(um)));
-  const float up = ldexpf(1.f, ex), down = ldexpf(1.f, -ex);
+  if (um >= 1.17549435e-38f && um < INFINITY) ex = max(-60, min(60, 14 - exp2_floor(um)));
+  const float up = pow2i(ex), down = pow2i(-ex);
   uint32_t Au[KU][4];
   {
     __half hv[NU][2][2];   // [q][row][hi, lo]
@@ -393,48 +373,58 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       Au[u][3] = h2u(__halves2half2(v[2][1], v[3][1]));
     }
   }
-  // accumulator = up * gamma_P S~0 (codes of this lane's fragments times scales); += U^^T K
+  // this warp's initialisation factors in fragment order: up gamma_P s_j (COL)
+  WarpTab<D>& wt = sm.wt[w];
+  if (col) {
+    const float gp = gP * up;
+    for (int e = lane; e < KS * 4; e += 32) {
+      const int ks = e >> 2, tt = e & 3;
+      float f[4];
+#pragma unroll
+      for (int pos = 0; pos < 4; ++pos) f[pos] = gp * sm.sc[jof<D, BITS>(tt, ks, pos)];
+      wt.f[ks][tt] = make_float4(f[0], f[1], f[2], f[3]);
+    }
+    __syncwarp();
+  }
+  const float fr0 = up * gP * sm.sc[i0], fr1 = up * gP * sm.sc[i1];
+  // accumulator: up gamma_P S~0 (the lane's own code fragments), then += U^^T K.
+  // Tile 2ks + hs, element e of lane (g, t) is key channel jof(t, ks, 2hs + e).
   float acc[NT][4];
-  const float fr0 = sm.rowv[i0] * up, fr1 = sm.rowv[i1] * up;
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     const float2 c0 = __half22float2(u2h(Af[ks][0])), c1 = __half22float2(u2h(Af[ks][1]));
     const float2 c2 = __half22float2(u2h(Af[ks][2])), c3 = __half22float2(u2h(Af[ks][3]));
+    float2 fa, fb, fc, fd;   // factors of c0 (row g, pos 0/1), c1 (row g+8), c2 (row g, pos 2/3), c3
     if (col) {
-      const float4 f = *reinterpret_cast<const float4*>(&sm.F[ks][t][0]);
-      const float f0 = f.x * up, f1 = f.y * up, f2 = f.z * up, f3 = f.w * up;
-      acc[2 * ks][0] = c0.x * f0; acc[2 * ks][1] = c0.y * f1;
-      acc[2 * ks][2] = c1.x * f0; acc[2 * ks][3] = c1.y * f1;
-      acc[2 * ks + 1][0] = c2.x * f2; acc[2 * ks + 1][1] = c2.y * f3;
-      acc[2 * ks + 1][2] = c3.x * f2; acc[2 * ks + 1][3] = c3.y * f3;
+      const float4 f = wt.f[ks][t];
+      fa = fb = make_float2(f.x, f.y);
+      fc = fd = make_float2(f.z, f.w);
     } else {
-      acc[2 * ks][0] = c0.x * fr0; acc[2 * ks][1] = c0.y * fr0;
-      acc[2 * ks][2] = c1.x * fr1; acc[2 * ks][3] = c1.y * fr1;
-      acc[2 * ks + 1][0] = c2.x * fr0; acc[2 * ks + 1][1] = c2.y * fr0;
-      acc[2 * ks + 1][2] = c3.x * fr1; acc[2 * ks + 1][3] = c3.y * fr1;
+      fa = fc = make_float2(fr0, fr0);
+      fb = fd = make_float2(fr1, fr1);
     }
+    const float2 v0 = __fmul2_rn(c0, fa), v1 = __fmul2_rn(c1, fb);
+    const float2 v2 = __fmul2_rn(c2, fc), v3 = __fmul2_rn(c3, fd);
+    acc[2 * ks][0] = v0.x; acc[2 * ks][1] = v0.y; acc[2 * ks][2] = v1.x; acc[2 * ks][3] = v1.y;
+    acc[2 * ks + 1][0] = v2.x; acc[2 * ks + 1][1] = v2.y; acc[2 * ks + 1][2] = v3.x; acc[2 * ks + 1][3] = v3.y;
 #pragma unroll
-    for (int hs = 0; hs < 2; ++hs) {
-      const int tile = 2 * ks + hs;
-      const int j = jof<D, BITS>(g >> 1, ks, 2 * hs + (g & 1));
+    for (int hs = 0; hs < 2; ++hs)
 #pragma unroll
       for (int u = 0; u < KU; ++u) {
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sm.bk[j][16 * u + 2 * t]);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sm.bk[j][16 * u + 2 * t + 8]);
-        mma16816(acc[tile], Au[u], b0, b1);
+        const uint2 bb = sm.bkf[2 * ks + hs][u][g][t];
+        mma16816(acc[2 * ks + hs], Au[u], bb.x, bb.y);
       }
-    }
   }
 
   // ---- absmax ----------------------------------------------------------------
   if (col) {
     float v[2 * NT];
 #pragma unroll
-    for (int tile = 0; tile < NT; ++tile) {
-      v[2 * tile] = max_nan(fabsf(acc[tile][0]), fabsf(acc[tile][2]));
-      v[2 * tile + 1] = max_nan(fabsf(acc[tile][1]), fabsf(acc[tile][3]));
+    for (int tau = 0; tau < NT; ++tau) {
+      v[2 * tau] = max_nan(fabsf(acc[tau][0]), fabsf(acc[tau][2]));
+      v[2 * tau + 1] = max_nan(fabsf(acc[tau][1]), fabsf(acc[tau][3]));
     }
-    // transpose-reduce over the 8 row lanes (lane bits 4, 3, 2): 2*NT -> 2*NT/8 values
+    // transpose-reduce over the 8 row lanes (lane bits 4, 3, 2)
 #pragma unroll
     for (int c = 2 * NT; c > 2 * NT / 8; c >>= 1) {
       const int o = c == 2 * NT ? 16 : (c == NT ? 8 : 4);
@@ -446,20 +436,19 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
         v[k] = max_nan(keep, __shfl_xor_sync(FULL, send, o));
       }
     }
-    // lane keeps value indices 4g + k (k < 2NT/8 = D/32): tile 2g + (k >> 1), column 2t + (k & 1)
+    // the lane keeps value indices (2NT/8) g + k (tile idx >> 1, element idx & 1)
 #pragma unroll
     for (int k = 0; k < 2 * NT / 8; ++k) {
       const int idx = (2 * NT / 8) * g + k;
-      const int tile = idx >> 1, e = idx & 1;
-      const int j = jof<D, BITS>(t, tile >> 1, 2 * (tile & 1) + e);
-      sm.colmax[w][j] = v[k] * down;
+      const int tau = idx >> 1;
+      sm.colmax[w][jof<D, BITS>(t, tau >> 1, 2 * (tau & 1) + (idx & 1))] = v[k] * down;
     }
   } else {
     float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-    for (int tile = 0; tile < NT; ++tile) {
-      m0 = max_nan(m0, max_nan(fabsf(acc[tile][0]), fabsf(acc[tile][1])));
-      m1 = max_nan(m1, max_nan(fabsf(acc[tile][2]), fabsf(acc[tile][3])));
+    for (int tau = 0; tau < NT; ++tau) {
+      m0 = max_nan(m0, max_nan(fabsf(acc[tau][0]), fabsf(acc[tau][1])));
+      m1 = max_nan(m1, max_nan(fabsf(acc[tau][2]), fabsf(acc[tau][3])));
     }
 #pragma unroll
     for (int off = 1; off <= 2; off <<= 1) {
@@ -467,19 +456,19 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       m1 = max_nan(m1, __shfl_xor_sync(FULL, m1, off));
     }
     if (t == 0) {
-      bool ovf = false;
       const float a0 = m0 * down, a1 = m1 * down;
       const GroupScale s0 = group_scale(a0, isfinite(a0), qmax, p.flags);
       const GroupScale s1 = group_scale(a1, isfinite(a1), qmax, p.flags);
-      ovf = !isfinite(a0) || !isfinite(a1) ||
-            (s0.bits == 0x7BFF && a0 / qmax > 65504.f) || (s1.bits == 0x7BFF && a1 / qmax > 65504.f);
+      const bool bad = !isfinite(a0) || !isfinite(a1) ||
+                       (s0.bits == 0x7BFF && a0 / qmax > 65504.f) ||
+                       (s1.bits == 0x7BFF && a1 / qmax > 65504.f);
       rsc[i0] = s0.bits;
       rsc[i1] = s1.bits;
-      sm.rowq[i0] = s0.sf > 0.f ? 1.f / s0.sf : 0.f;
-      sm.rowq[i1] = s1.sf > 0.f ? 1.f / s1.sf : 0.f;
-      sm.rows[i0] = s0.sf;
-      sm.rows[i1] = s1.sf;
-      if (ovf) sm.slow = 1;
+      sm.qf[i0] = s0.sf > 0.f ? __frcp_rn(s0.sf) : 0.f;
+      sm.qf[i1] = s1.sf > 0.f ? __frcp_rn(s1.sf) : 0.f;
+      sm.sfv[i0] = s0.sf;
+      sm.sfv[i1] = s1.sf;
+      if (bad) sm.slow = 1;
     }
   }
   __syncthreads();
@@ -490,10 +479,8 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       for (int ww = 0; ww < C::RB; ++ww) a = max_nan(a, sm.colmax[ww][j]);
       const GroupScale s = group_scale(a, isfinite(a), qmax, p.flags);
       rsc[j] = s.bits;
-      int tt, ks, pos;
-      kslot_of<D, BITS>(j, tt, ks, pos);
-      sm.qfr[ks][tt][pos] = s.sf > 0.f ? 1.f / s.sf : 0.f;
-      sm.sfr[ks][tt][pos] = s.sf;
+      sm.qf[j] = s.sf > 0.f ? __frcp_rn(s.sf) : 0.f;
+      sm.sfv[j] = s.sf;
       if (!isfinite(a) || (s.bits == 0x7BFF && a / qmax > 65504.f)) sm.slow = 1;
     }
     __syncthreads();
@@ -501,61 +488,75 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 
   // ---- encode and store this warp's rows ------------------------------------
   const bool slow = sm.slow != 0;
-  uint32_t hm[KS][2][2];   // [ks][tile half][row] f16x2 magic pairs
+  if (col) {
+    for (int e = lane; e < KS * 4; e += 32) {
+      const int ks = e >> 2, tt = e & 3;
+      float f[4];
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    float q0, q1, q2, q3, qa, qb;   // per column (COL) or per row (ROW)
-    if (col) {
-      const float4 qq = *reinterpret_cast<const float4*>(slow ? &sm.sfr[ks][t][0] : &sm.qfr[ks][t][0]);
-      q0 = qq.x; q1 = qq.y; q2 = qq.z; q3 = qq.w;
-      qa = qb = 0.f;
-    } else {
-      qa = slow ? sm.rows[i0] : sm.rowq[i0];
-      qb = slow ? sm.rows[i1] : sm.rowq[i1];
-      q0 = q1 = q2 = q3 = 0.f;
-    }
-#pragma unroll
-    for (int hs = 0; hs < 2; ++hs) {
-      const float* a = acc[2 * ks + hs];
-      const float ca = col ? (hs ? q2 : q0) : qa, cb = col ? (hs ? q3 : q1) : qa;
-      const float cc = col ? (hs ? q2 : q0) : qb, cd = col ? (hs ? q3 : q1) : qb;
-      if (!slow) {
-        hm[ks][hs][0] = magic_fast<BITS>(a[0], a[1], ca * down, cb * down);
-        hm[ks][hs][1] = magic_fast<BITS>(a[2], a[3], cc * down, cd * down);
-      } else {
-        hm[ks][hs][0] = magic_exact<BITS>(a[0] * down, a[1] * down, ca, cb);
-        hm[ks][hs][1] = magic_exact<BITS>(a[2] * down, a[3] * down, cc, cd);
+      for (int pos = 0; pos < 4; ++pos) {
+        const int j = jof<D, BITS>(tt, ks, pos);
+        f[pos] = slow ? sm.sfv[j] : sm.qf[j] * down;
       }
+      wt.q[ks][tt] = make_float4(f[0], f[1], f[2], f[3]);
     }
+    __syncwarp();
   }
-  constexpr int ROWB = D * BITS / 8;
+  const float qr0 = col ? 0.f : (slow ? sm.sfv[i0] : sm.qf[i0] * down);
+  const float qr1 = col ? 0.f : (slow ? sm.sfv[i1] : sm.qf[i1] * down);
+  auto encode_rows = [&](auto fast) {
+    // magic f16 pair of value (ks_a, pos_a) and (ks_b, pos_b) of row half rr;
+    // value (ks, pos) sits in tile 2ks + (pos >> 1), element pos & 1
+    auto mk = [&](int ksa, int pa, int ksb, int pb, int rr) -> uint32_t {
+      const float a = acc[2 * ksa + (pa >> 1)][2 * rr + (pa & 1)];
+      const float bq = acc[2 * ksb + (pb >> 1)][2 * rr + (pb & 1)];
+      float qa = rr ? qr1 : qr0, qb = qa;
+      if (col) {
+        qa = pick4(wt.q[ksa][t], pa);
+        qb = pick4(wt.q[ksb][t], pb);
+      }
+      if (decltype(fast)::value) return magic_fast<BITS>(a, bq, qa, qb);
+      return magic_exact<BITS>(a * down, bq * down, qa, qb);
+    };
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    uint8_t* row = rec + (size_t)(rr ? i1 : i0) * ROWB;
-    if (BITS == 4) {
-      constexpr int NW = D / 32;   // words per lane per row
-      uint32_t wd[NW];
+    for (int rr = 0; rr < 2; ++rr) {
+      uint8_t* row = rec + (size_t)(rr ? i1 : i0) * ROWB;
+      if (BITS == 4) {
+        // word m holds channels 8m + k of the lane's range: k-step 2m gives
+        // k = 0 (pos 0), 4 (pos 1), 1 (pos 2), 5 (pos 3); k-step 2m+1 gives k + 2
+        constexpr int NW = D / 32;
+        uint32_t wd[NW];
 #pragma unroll
-      for (int m = 0; m < NW; ++m)
-        wd[m] = pack_int4(hm[2 * m][0][rr], hm[2 * m][1][rr], hm[2 * m + 1][0][rr], hm[2 * m + 1][1][rr]);
-      uint8_t* dst = row + chunk_offset<D, 4>(t, 0);
-      if (NW == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      else if (NW == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1]);
-      else *reinterpret_cast<uint32_t*>(dst) = wd[0];
-    } else {
-      constexpr int WPC = D / 32;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t wd[WPC];
-#pragma unroll
-        for (int m = 0; m < WPC; ++m) wd[m] = pack_int8(hm[c * WPC + m][0][rr], hm[c * WPC + m][1][rr]);
-        uint8_t* dst = row + chunk_offset<D, 8>(t, c);
-        if (WPC == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-        else if (WPC == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1]);
+        for (int m = 0; m < NW; ++m) {
+          const int ka = 2 * m, kb = 2 * m + 1;
+          const uint32_t E = prmt(mk(ka, 0, kb, 0, rr), mk(ka, 1, kb, 1, rr), 0x6420u);  // k 0 2 4 6
+          const uint32_t O = prmt(mk(ka, 2, kb, 2, rr), mk(ka, 3, kb, 3, rr), 0x6420u);  // k 1 3 5 7
+          wd[m] = (E | (O << 4)) ^ 0x88888888u;
+        }
+        uint8_t* dst = row + chunk_offset<D, 4>(t, 0);
+        if (NW == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        else if (NW == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1]);
         else *reinterpret_cast<uint32_t*>(dst) = wd[0];
+      } else {
+        // k-step ks covers channels base + pos of one code word
+        constexpr int WPC = D / 32;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t wd[WPC];
+#pragma unroll
+          for (int m = 0; m < WPC; ++m) {
+            const int ks = c * WPC + m;
+            wd[m] = prmt(mk(ks, 0, ks, 1, rr), mk(ks, 2, ks, 3, rr), 0x6420u) ^ 0x80808080u;
+          }
+          uint8_t* dst = row + chunk_offset<D, 8>(t, c);
+          if (WPC == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          else if (WPC == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1]);
+          else *reinterpret_cast<uint32_t*>(dst) = wd[0];
+        }
       }
     }
-  }
+  };
+  if (!slow) encode_rows(std::true_type{});
+  else encode_rows(std::false_type{});
   if (tid == 0) p.fill[head] = 0;
 }
 
@@ -567,19 +568,15 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
   Smem<D, BF16, PMAX>& sm = *reinterpret_cast<Smem<D, BF16, PMAX>*>(smem_raw);
   const int tid = threadIdx.x;
   const int n_heads = p.B * p.H;
-  // zero the operand slots that stay unused (tokens >= P, padding segments)
-  {
-    uint32_t* z = &sm.bx[0][0][0][0][0];
+  {   // operand columns that stay unused (vectors >= P) must read as zero
+    uint32_t* z = reinterpret_cast<uint32_t*>(&sm.bx[0][0][0][0]);
     for (int i = tid; i < (int)(sizeof(sm.bx) / 4); i += C::THREADS) z[i] = 0u;
-    uint32_t* zb = reinterpret_cast<uint32_t*>(&sm.bk[0][0]);  // whole rows incl. padding
-    for (int i = tid; i < (int)(sizeof(sm.bk) / 4); i += C::THREADS) zb[i] = 0u;
   }
   if (tid == 0) {
     mbar_init(&sm.bar[0], 1);
     mbar_init(&sm.bar[1], 1);
     fence_mbar_init();
     sm.slow = 0;
-    sm.abort_ = 0;
     const int first = find_full(p, blockIdx.x, gridDim.x, n_heads);
     sm.next_head = first;
     if (first < n_heads) issue_head<D, BF16, PMAX>(p, first, sm, 0);
@@ -598,11 +595,9 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     const bool ok = mbar_wait_bounded(&sm.bar[s], parity[s], p.flags);
     parity[s] ^= 1u;
     if (__syncthreads_or(!ok)) {
-      // a copy did not land in time: give the in-flight copies a bounded
-      // second chance to finish before this block's shared memory goes away
-      if (tid == 0) {
-        mbar_wait_bounded(&sm.bar[s ^ 1], parity[s ^ 1], nullptr);
-      }
+      // a copy did not land in time: give the other in-flight copy a bounded
+      // chance to finish before this block's shared memory is released
+      if (tid == 0) mbar_wait_bounded(&sm.bar[s ^ 1], parity[s ^ 1], nullptr);
       __syncthreads();
       return;
     }

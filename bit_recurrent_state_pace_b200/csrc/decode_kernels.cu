@@ -39,6 +39,8 @@ template <int D>
 struct alignas(16) WarpScratch {
   uint8_t dig[4][D];               // digits 0..2 of the right-hand side, row 3 = zeros
   float y[D];                      // S~0 q^ by row, before the row scale
+  float A[PACE_MAX_PERIOD * PACE_MAX_PERIOD];   // period end: A[t][s]
+  float gsb[3][PACE_MAX_PERIOD];                // period end: gamma_s, gamma_{P/s}, beta_s
 };
 
 // Lane L ends with the warp-wide sum of value index (L mod V).
@@ -67,7 +69,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
                                             const void* __restrict__ alpha,
                                             const void* __restrict__ beta, float* __restrict__ o,
                                             WarpScratch<D>& scr, int lane) {
-  constexpr int EPL = D / 32, RB = D / 16, KS = D / 16, PF = 2;
+  constexpr int EPL = D / 32, RB = D / 16, PF = 2;
   constexpr int ESZ = BF16 ? 2 : 4;
   const int g = lane >> 2, t = lane & 3;
   const int h = head % p.H, b = head / p.H;
@@ -170,6 +172,13 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
       else if (tt == n - 1) G = tot;
     }
     acol[tt] = (tt > lane && tt < n) ? bt * run * G : 0.f;
+  }
+  if (n == P && lane < PMAX) {         // kept for the period-end factors (step 12)
+#pragma unroll
+    for (int tt = 0; tt < PMAX; ++tt) scr.A[tt * PMAX + lane] = acol[tt];
+    scr.gsb[0][lane] = gcum;
+    scr.gsb[1][lane] = suf;
+    scr.gsb[2][lane] = be;
   }
   // 6. backward substitution (I + A^T) y = w, lane-parallel over s
   float acc = w_s;
@@ -356,7 +365,31 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     ra.store(abp, 0);
     rb2.store(abp, 1);
   }
-  if (lane < n - 1) const_cast<float*>(gram_head)[(n - 1) * P + lane] = tot;
+  if (n < P && lane < n - 1) const_cast<float*>(gram_head)[(n - 1) * P + lane] = tot;
+
+  // 12. period end (n == P): replace the Gram block by the commit's chunk-form
+  //     factors W[t][s] = gamma_{P/t} T[t][s] beta_s, T = (I + A)^{-1} (lane s
+  //     solves column s by forward substitution), followed by gamma_s
+  if (n == P) {
+    __syncwarp();
+    float Tc[PMAX];
+#pragma unroll
+    for (int tt = 0; tt < PMAX; ++tt) {
+      float a2 = 0.f;
+#pragma unroll
+      for (int r = 0; r < tt; ++r)
+        if (r >= lane) a2 = fmaf(scr.A[tt * PMAX + r], Tc[r], a2);
+      Tc[tt] = tt == lane ? 1.f : (tt > lane ? -a2 : 0.f);
+    }
+    float* gw = const_cast<float*>(gram_head);
+    if (lane < P) {
+      const float bs = scr.gsb[2][lane];
+#pragma unroll
+      for (int tt = 0; tt < PMAX; ++tt)
+        if (tt < P) gw[tt * P + lane] = scr.gsb[1][tt] * Tc[tt] * bs;
+      gw[P * P + lane] = scr.gsb[0][lane];
+    }
+  }
   __syncwarp();
   if (lane == 0) p.fill[head] = n;
 }
