@@ -316,8 +316,8 @@ def run_pace(args, rank: int, world: int):
     else:
         ach, traffic = com_gbs, ncu_traffic("commit", digest)
 
-    units = BH * P * args.steps * world
-    value = units / (elapsed_ms * 1e-3)
+    from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+    value = aggregate_rate(BH * P * args.steps, world, elapsed_ms)
 
     # ---- bf16-state comparison path (unquantised, same shape)
     compare = None
@@ -409,27 +409,22 @@ def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev):
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world, dev)
-    units = w.B * w.H * P * args.e2e_steps * world
-    return {"value": units / (ms * 1e-3), "unit": "head-tokens/s", "h2d_bytes_per_step": h2d,
+    from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+    return {"value": aggregate_rate(w.B * w.H * P * args.e2e_steps, world, ms),
+            "unit": "head-tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from bit_recurrent_state_pace_b200.ranks import barrier as _barrier
+    _barrier(world)
 
 
 def max_over_ranks(x: float, world: int, dev):
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from bit_recurrent_state_pace_b200.ranks import max_over_ranks as _max
+    return _max(x, world, dev)
 
 
 def main():

@@ -240,8 +240,11 @@ class PacePool:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
-            pace_destroy_pool(h)
+        if h and pace_destroy_pool is not None:   # module globals are gone at interpreter exit
+            try:
+                pace_destroy_pool(h)
+            except Exception:
+                pass
             self.handle = None
 
     # layout helpers -----------------------------------------------------
