@@ -17,13 +17,21 @@
 // product (S~0 q^) per token.
 //
 // Design (B200): one warp owns one head at a time (no block barriers); heads
-// are strided over a persistent grid.  The codes stream from HBM with
-// coalesced 128-bit non-allocating loads straight into the A-fragment
-// registers of mma.sync m16n8k16 (f16 codes exact, fp32 accumulation; the
-// right-hand side q^ is split hi + lo in f16), prefetched two 16-row blocks
-// ahead.  The small n x n chunk algebra runs lane-parallel over tokens with
-// warp shuffles; k.k dot products of earlier buffered tokens are cached in
-// the buffer's Gram region, so each step computes only the 2n-1 new ones.
+// are strided over a persistent grid.
+//  * Staging: everything of a head except its codes -- q, k, v of the token,
+//    the fp16 scales, the n-1 buffered (k, v) rows, their gates and Gram
+//    block -- is brought into the warp's shared-memory stage by 1-D bulk
+//    copies (TMA, no multicast) one head ahead, completing on a per-stage
+//    mbarrier; the chunk algebra then reads on-chip data only.
+//  * State stream: the codes go from HBM (L2-prefetched one head ahead) with
+//    coalesced 128-bit non-allocating loads straight into the A fragments of
+//    the int8 tensor cores (mma.sync m16n8k32, s8 x s8 for INT8 codes; INT4
+//    nibbles widened to offset bytes, u8 x s8), two 16-row blocks ahead; the
+//    right-hand side q^ (times the column scales) enters as 22-bit fixed
+//    point split into three base-256 digits, so the products are exact int32.
+//  * The small n x n chunk algebra runs lane-parallel over tokens with warp
+//    shuffles; k.k dot products of earlier buffered tokens are cached in the
+//    buffer's Gram block, so each step computes only the 2n-1 new ones.
 #include "frag.cuh"
 #include "tma.cuh"
 
@@ -41,6 +49,20 @@ struct alignas(16) WarpScratch {
   float y[D];                      // S~0 q^ by row, before the row scale
   float A[PACE_MAX_PERIOD * PACE_MAX_PERIOD];   // period end: A[t][s]
   float gsb[3][PACE_MAX_PERIOD];                // period end: gamma_s, gamma_{P/s}, beta_s
+};
+
+// One warp's shared-memory stage for one head (byte offsets, all 16-aligned).
+template <int D, bool BF16, int PMAX>
+struct Stage {
+  static constexpr int ESZ = BF16 ? 2 : 4;
+  static constexpr int Q = 0, K = D * ESZ, V = 2 * D * ESZ;     // token inputs
+  static constexpr int SC = 3 * D * ESZ;                          // fp16 scales [D]
+  static constexpr int KV = SC + 2 * D;                           // rows [PMAX-1][k | v]
+  static constexpr int AB = KV + (PMAX - 1) * 2 * D * ESZ;        // gates [PMAX][2]
+  static constexpr int G = AB + (2 * PMAX * ESZ + 15) / 16 * 16;  // Gram [PMAX][PMAX] + [PMAX]
+  static constexpr int BYTES = G + (4 * PMAX * (PMAX + 1) + 15) / 16 * 16;
+  // two stages (copies one head ahead) while 8 warps fit twice per SM
+  static constexpr int N = 2 * 8 * 2 * BYTES <= 160 * 1024 ? 2 : 1;
 };
 
 // Lane L ends with the warp-wide sum of value index (L mod V).
@@ -68,7 +90,8 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
                                             const void* __restrict__ k, const void* __restrict__ v,
                                             const void* __restrict__ alpha,
                                             const void* __restrict__ beta, float* __restrict__ o,
-                                            WarpScratch<D>& scr, int lane) {
+                                            WarpScratch<D>& scr, const uint8_t* stg, int lane) {
+  using ST = Stage<D, BF16, PMAX>;
   constexpr int EPL = D / 32, RB = D / 16, PF = 2;
   constexpr int ESZ = BF16 ? 2 : 4;
   const int g = lane >> 2, t = lane & 3;
@@ -82,12 +105,12 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   for (int r = 0; r < PF; ++r) rbuf[r].load(rec, r, g, t);
 
   // 2. this token's inputs and the head's scales (lane holds elements EPL*lane..)
-  const size_t e0 = (size_t)head * D + (size_t)EPL * lane;
+  const size_t e0 = (size_t)EPL * lane;
   Raw<EPL, BF16> k_raw, v_raw;
-  k_raw.load(k, e0);
-  v_raw.load(v, e0);
+  k_raw.load(stg + ST::K, e0);
+  v_raw.load(stg + ST::V, e0);
   float qf[EPL], kf[EPL], vf[EPL], sc[EPL];
-  load_f<EPL, BF16>(q, e0, qf);
+  load_f<EPL, BF16>(stg + ST::Q, e0, qf);
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
     kf[e] = k_raw.get(e);
@@ -97,7 +120,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   const float b_n = load_io(beta, head, BF16 ? PACE_IO_BF16 : PACE_IO_F32);
   {
     Raw<EPL, true> s_raw;   // fp16 scales share the bf16 byte layout
-    s_raw.load(rec + code_bytes(D, D, BITS), (size_t)EPL * lane);
+    s_raw.load(stg + ST::SC, (size_t)EPL * lane);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       const uint32_t x = s_raw.w[e >> 1];
@@ -108,6 +131,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   // 3. dot products with the buffered keys: k_n.k_s and q.k_s
   const size_t row_elems = 2 * (size_t)D;
   const uint8_t* kv_head = p.kv + (size_t)head * P * row_elems * ESZ;
+  const uint8_t* kv_stg = stg + ST::KV;
   float part[2 * PMAX];
 #pragma unroll
   for (int i = 0; i < 2 * PMAX; ++i) part[i] = 0.f;
@@ -115,7 +139,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   for (int s = 0; s < PMAX; ++s) {
     if (s < n - 1) {
       float ks[EPL];
-      load_f<EPL, BF16>(kv_head, s * row_elems + (size_t)EPL * lane, ks);
+      load_f<EPL, BF16>(kv_stg, s * row_elems + (size_t)EPL * lane, ks);
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
         part[s] = fmaf(kf[e], ks[e], part[s]);
@@ -134,7 +158,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   const uint8_t* ab_head = p.ab + (size_t)head * p.ab_stride;
   if (lane < n - 1) {
     Raw<2, BF16> ab;
-    ab.load(ab_head, (size_t)lane * 2);
+    ab.load(stg + ST::AB, (size_t)lane * 2);
     al = ab.get(0);
     be = ab.get(1);
   } else if (lane == n - 1) {
@@ -168,7 +192,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     float G = 0.f;
     if (tt > lane) {
       run *= at;
-      if (tt < n - 1) G = gram_head[tt * P + lane];
+      if (tt < n - 1) G = reinterpret_cast<const float*>(stg + ST::G)[tt * P + lane];
       else if (tt == n - 1) G = tot;
     }
     acol[tt] = (tt > lane && tt < n) ? bt * run * G : 0.f;
@@ -206,8 +230,8 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
       const float zs = __shfl_sync(FULL, z, s);
       float ks[EPL], vs[EPL];
       if (s < n - 1) {
-        load_f<EPL, BF16>(kv_head, s * row_elems + (size_t)EPL * lane, ks);
-        load_f<EPL, BF16>(kv_head, s * row_elems + D + (size_t)EPL * lane, vs);
+        load_f<EPL, BF16>(kv_stg, s * row_elems + (size_t)EPL * lane, ks);
+        load_f<EPL, BF16>(kv_stg, s * row_elems + D + (size_t)EPL * lane, vs);
       } else {
 #pragma unroll
         for (int e = 0; e < EPL; ++e) { ks[e] = kf[e]; vs[e] = vf[e]; }
@@ -394,51 +418,106 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   if (lane == 0) p.fill[head] = n;
 }
 
+// Bulk-copy head `head`'s staged inputs into `stg` (lane 0 only): q, k, v, the
+// scales, and -- when `fill` tokens (0 < fill < P) are buffered -- its rows,
+// gates and Gram block.  Completes on `bar` with the exact byte count.
+template <int D, bool BF16, int PMAX>
+__device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill, const void* q,
+                                            const void* k, const void* v, uint8_t* stg,
+                                            uint64_t* bar) {
+  using ST = Stage<D, BF16, PMAX>;
+  constexpr uint32_t IO = D * ST::ESZ;
+  const int h = head % p.H, b = head / p.H;
+  const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
+  const bool rows = fill > 0 && fill < p.P;
+  const uint32_t kv_bytes = rows ? (uint32_t)fill * 2 * IO : 0u;
+  const uint32_t bytes = 3 * IO + 2 * D + (rows ? kv_bytes + p.ab_stride + p.gram_stride : 0u);
+  fence_proxy_async_smem();
+  mbar_arrive_expect_tx(bar, bytes);
+  tma_load_1d(stg + ST::Q, reinterpret_cast<const uint8_t*>(q) + (size_t)head * IO, IO, bar);
+  tma_load_1d(stg + ST::K, reinterpret_cast<const uint8_t*>(k) + (size_t)head * IO, IO, bar);
+  tma_load_1d(stg + ST::V, reinterpret_cast<const uint8_t*>(v) + (size_t)head * IO, IO, bar);
+  tma_load_1d(stg + ST::SC, rec + code_bytes(D, D, p.bits[h]), 2 * D, bar);
+  if (rows) {
+    tma_load_1d(stg + ST::KV, p.kv + (size_t)head * p.P * 2 * IO, kv_bytes, bar);
+    tma_load_1d(stg + ST::AB, p.ab + (size_t)head * p.ab_stride, p.ab_stride, bar);
+    tma_load_1d(stg + ST::G, p.gram + (size_t)head * p.gram_stride, p.gram_stride, bar);
+  }
+}
+
 template <int D, bool BF16, int PMAX>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_step_kernel(PoolDev p, const void* __restrict__ q, const void* __restrict__ k,
                        const void* __restrict__ v, const void* __restrict__ alpha,
                        const void* __restrict__ beta, float* __restrict__ o) {
-  __shared__ WarpScratch<D> scratch[kWarpsPerBlock];
+  using ST = Stage<D, BF16, PMAX>;
+  constexpr int NS = ST::N;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  WarpScratch<D>& scr = scratch[wib];
+  uint8_t* stages = smem_raw + (size_t)wib * NS * ST::BYTES;
+  WarpScratch<D>& scr =
+      reinterpret_cast<WarpScratch<D>*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES)[wib];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES +
+                                              kWarpsPerBlock * sizeof(WarpScratch<D>)) + NS * wib;
   for (int i = lane; i < D; i += 32) scr.dig[3][i] = 0;
-  __syncwarp();
   const int n_heads = p.B * p.H;
   const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
-  const int n_warps = gridDim.x * kWarpsPerBlock;
-  constexpr int ESZ = BF16 ? 2 : 4;
-  int fill_next = 0;
-  if (lane == 0 && warp0 < n_heads) fill_next = p.fill[warp0];
-  for (int head = warp0; head < n_heads; head += n_warps) {
-    int nprev = __shfl_sync(FULL, fill_next, 0);
-    // start the next head of this warp on its way into L2: its record and
-    // inputs now, its buffered rows once its fill count is known
-    const int nh = head + n_warps;
-    if (lane == 0 && nh < n_heads) {
-      const int hh = nh % p.H;
-      prefetch_l2(p.state + (size_t)(nh / p.H) * p.slot_stride + p.rec_off[hh],
-                  (uint32_t)record_bytes(D, D, p.bits[hh], D));
-      prefetch_l2(reinterpret_cast<const uint8_t*>(q) + (size_t)nh * D * ESZ, D * ESZ);
-      prefetch_l2(reinterpret_cast<const uint8_t*>(k) + (size_t)nh * D * ESZ, D * ESZ);
-      prefetch_l2(reinterpret_cast<const uint8_t*>(v) + (size_t)nh * D * ESZ, D * ESZ);
-      fill_next = p.fill[nh];
+  const int W = gridDim.x * kWarpsPerBlock;
+  // lane 0 keeps the fill counts of the current head and the next one
+  int f_cur = 0, f_nxt = 0;
+  if (lane == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
+    fence_mbar_init();
+    if (warp0 < n_heads) {
+      f_cur = p.fill[warp0];
+      if (NS == 2) issue_stage<D, BF16, PMAX>(p, warp0, f_cur, q, k, v, stages, &bar[0]);
+      f_nxt = warp0 + W < n_heads ? p.fill[warp0 + W] : 0;
     }
+  }
+  __syncwarp();
+  uint32_t parity = 0u;   // bit i: phase of stage i to wait for
+  int s = 0;
+  for (int head = warp0; head < n_heads; head += W) {
+    const int nh = head + W;
+    if (lane == 0) {
+      if (NS == 2) {
+        if (nh < n_heads)
+          issue_stage<D, BF16, PMAX>(p, nh, f_nxt, q, k, v, stages + (s ^ 1) * ST::BYTES, &bar[s ^ 1]);
+      } else {
+        issue_stage<D, BF16, PMAX>(p, head, f_cur, q, k, v, stages, &bar[0]);
+      }
+      if (nh < n_heads) {   // the next head's codes on their way into L2
+        const int hh = nh % p.H;
+        prefetch_l2(p.state + (size_t)(nh / p.H) * p.slot_stride + p.rec_off[hh],
+                    (uint32_t)record_bytes(D, D, p.bits[hh], D));
+      }
+    }
+    const int nprev = __shfl_sync(FULL, f_cur, 0);
+    if (lane == 0) {
+      f_cur = f_nxt;
+      f_nxt = nh + W < n_heads ? p.fill[nh + W] : 0;
+    }
+    const bool ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, lane == 0 ? p.flags : nullptr);
+    parity ^= 1u << s;
+    if (!__all_sync(FULL, ok)) {
+      // a copy did not land in time: let the other stage's copy finish (bounded)
+      // before this warp stops using its shared memory
+      if (NS == 2 && nh < n_heads) mbar_wait_bounded(&bar[s ^ 1], (parity >> (s ^ 1)) & 1u, nullptr);
+      return;
+    }
+    const uint8_t* stg = stages + s * ST::BYTES;
+    if (NS == 2) s ^= 1;
     if (nprev < 0 || nprev >= p.P) {
       if (lane == 0) atomicOr(p.flags, PACE_FLAG_BUFFER_FULL);
       for (int i = lane; i < D; i += 32) o[(size_t)head * D + i] = __int_as_float(0x7fc00000);
+      __syncwarp();
       continue;
     }
     const int n = nprev + 1;
     if (p.bits[head % p.H] == 4)
-      decode_head<D, BF16, PMAX, 4>(p, head, n, q, k, v, alpha, beta, o, scr, lane);
+      decode_head<D, BF16, PMAX, 4>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
     else
-      decode_head<D, BF16, PMAX, 8>(p, head, n, q, k, v, alpha, beta, o, scr, lane);
-    if (lane == 0 && nh < n_heads && fill_next > 0 && fill_next < p.P) {
-      prefetch_l2(p.kv + (size_t)nh * p.P * 2 * D * ESZ, (uint32_t)(fill_next * 2 * D * ESZ));
-      prefetch_l2(p.ab + (size_t)nh * p.ab_stride, p.ab_stride);
-      prefetch_l2(p.gram + (size_t)nh * p.gram_stride, p.gram_stride);
-    }
+      decode_head<D, BF16, PMAX, 8>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
   }
 }
 
@@ -458,11 +537,17 @@ int sm_count() {
 template <int D, bool BF16, int PMAX>
 cudaError_t launch_t(const PoolDev& p, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
+  using ST = Stage<D, BF16, PMAX>;
+  const size_t smem = (size_t)kWarpsPerBlock * (ST::N * ST::BYTES + sizeof(WarpScratch<D>) +
+                                                ST::N * sizeof(uint64_t));
+  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   const long heads = (long)p.B * p.H;
   long blocks = (heads + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const long cap = 2L * sm_count();
   if (blocks > cap) blocks = cap;
-  decode_step_kernel<D, BF16, PMAX><<<(unsigned)blocks, kThreads, 0, st>>>(p, q, k, v, alpha, beta, o);
+  decode_step_kernel<D, BF16, PMAX><<<(unsigned)blocks, kThreads, smem, st>>>(p, q, k, v, alpha, beta, o);
   return cudaGetLastError();
 }
 
