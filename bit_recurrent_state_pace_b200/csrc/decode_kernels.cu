@@ -17,7 +17,7 @@
 // product (S~0 q^) per token.
 //
 // Design (B200): one warp owns one head at a time (no block barriers); heads
-// are strided over a persistent grid.
+// are strided over a persistent grid in work order (4-bit heads first).
 //  * Staging: everything of a head except its codes -- q, k, v of the token,
 //    the fp16 scales, the n-1 buffered (k, v) rows, their gates and Gram
 //    block -- is brought into the warp's shared-memory stage by 1-D bulk
@@ -327,10 +327,15 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   const int cB = t == 0 ? corr[1] : 0;
 
   // 9. y = S~0 (codes) x b on the int8 tensor cores (exact int32), 16 rows at a time
+  // (unrolled by the prefetch depth only: a smaller loop body keeps the
+  // instruction cache warm for the 16 warps of an SM)
+#pragma unroll 1
+  for (int r0 = 0; r0 < RB; r0 += PF)
 #pragma unroll
-  for (int r = 0; r < RB; ++r) {
-    RowBlock<D, BITS> cur = rbuf[r % PF];
-    if (r + PF < RB) rbuf[r % PF].load(rec, r + PF, g, t);
+  for (int rr = 0; rr < PF; ++rr) {
+    const int r = r0 + rr;
+    RowBlock<D, BITS> cur = rbuf[rr];
+    if (r + PF < RB) rbuf[rr].load(rec, r + PF, g, t);
     int d[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
@@ -469,16 +474,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
     if (warp0 < n_heads) {
-      f_cur = p.fill[warp0];
-      if (NS == 2) issue_stage<D, BF16, PMAX>(p, warp0, f_cur, q, k, v, stages, &bar[0]);
-      f_nxt = warp0 + W < n_heads ? p.fill[warp0 + W] : 0;
+      const int h0 = head_in_order(p, warp0);
+      f_cur = p.fill[h0];
+      if (NS == 2) issue_stage<D, BF16, PMAX>(p, h0, f_cur, q, k, v, stages, &bar[0]);
+      f_nxt = warp0 + W < n_heads ? p.fill[head_in_order(p, warp0 + W)] : 0;
     }
   }
   __syncwarp();
   uint32_t parity = 0u;   // bit i: phase of stage i to wait for
   int s = 0;
-  for (int head = warp0; head < n_heads; head += W) {
-    const int nh = head + W;
+  for (int it = warp0; it < n_heads; it += W) {
+    const int head = head_in_order(p, it);
+    const int nh = it + W < n_heads ? head_in_order(p, it + W) : n_heads;
     if (lane == 0) {
       if (NS == 2) {
         if (nh < n_heads)
@@ -495,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nprev = __shfl_sync(FULL, f_cur, 0);
     if (lane == 0) {
       f_cur = f_nxt;
-      f_nxt = nh + W < n_heads ? p.fill[nh + W] : 0;
+      f_nxt = it + 2 * W < n_heads ? p.fill[head_in_order(p, it + 2 * W)] : 0;
     }
     const bool ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, lane == 0 ? p.flags : nullptr);
     parity ^= 1u << s;

@@ -30,7 +30,21 @@ struct PoolDev {
   uint32_t* flags;            // status word
   uint32_t rec_off[PACE_MAX_HEADS];   // record offset of head h inside a slot
   uint8_t bits[PACE_MAX_HEADS];       // 4 or 8
+  uint8_t order[PACE_MAX_HEADS];      // head indices, the 4-bit heads first
+  int32_t H4;                         // number of 4-bit heads
 };
+
+// The i-th (slot, head) in work order: all 4-bit heads of every slot, then
+// all 8-bit ones, so that the warps of a launch run one code path at a time.
+__device__ __forceinline__ int head_in_order(const PoolDev& p, int i) {
+  const int n4 = p.B * p.H4;
+  if (i < n4) {
+    const int b = i / p.H4;
+    return b * p.H + p.order[i - b * p.H4];
+  }
+  const int h8 = p.H - p.H4, j = i - n4, b = j / h8;
+  return b * p.H + p.order[p.H4 + j - b * h8];
+}
 
 __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -146,6 +146,14 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
   dv.gram_stride = pace::gram_stride_bytes(desc->period);
   dv.fill = static_cast<int32_t*>(d_aux);
   dv.flags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(d_aux) + L.aux_bytes - 256);
+  {
+    int n4 = 0;
+    for (int h = 0; h < desc->num_heads; ++h)
+      if (desc->head_bits[h] == 4) dv.order[n4++] = (uint8_t)h;
+    dv.H4 = n4;
+    for (int h = 0; h < desc->num_heads; ++h)
+      if (desc->head_bits[h] != 4) dv.order[n4++] = (uint8_t)h;
+  }
   for (int h = 0; h < desc->num_heads; ++h) {
     dv.rec_off[h] = (uint32_t)L.rec_off[h];
     dv.bits[h] = desc->head_bits[h];
