@@ -67,7 +67,7 @@ struct Cfg {
   static constexpr int REC = (D * D + 2 * D + 15) / 16 * 16;   // largest record (INT8)
   static constexpr int KVB = PMAX * 2 * D * ESZ;
   static constexpr int ABB = (2 * PMAX * ESZ + 15) / 16 * 16;
-  static constexpr int GRB = (4 * PMAX * (PMAX + 1) + 15) / 16 * 16;
+  static constexpr int GRB = (4 * (PMAX * (PMAX + 1) + 2) + 15) / 16 * 16;
   static constexpr int SLOT = REC + KVB + ABB + GRB;
 };
 
@@ -185,89 +185,74 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   const uint16_t* s_sc = reinterpret_cast<const uint16_t*>(s_rec + code_bytes(D, D, BITS));
 
   // ---- phase 1: per-head operands ------------------------------------------
-  // W[s][s'] (P x P) and gamma_s (P) were left in the Gram block by the decode
-  // step that buffered the P-th token.
+  // W[s][s'] (P x P), gamma_s (P), max |k| and the largest stored scale were
+  // left in the Gram block by the decode step that buffered the P-th token.
   const float* W = s_gr;
   const float* gam = s_gr + P * P;
   const float gP = gam[P - 1];
   for (int j = tid; j < D; j += C::THREADS) sm.sc[j] = __half2float(__ushort_as_half(s_sc[j]));
+  // one power-of-two normalisation of the X operand for the whole head
+  const float bmax = col ? s_gr[P * P + P] * s_gr[P * P + P + 1] : s_gr[P * P + P];
+  int exx = 0;
+  if (bmax >= 1.17549435e-38f && bmax < INFINITY) exx = max(-120, min(120, 14 - exp2_floor(bmax)));
+  const float upx = pow2i(exx);
+  if (tid == 0) sm.xinv = pow2i(-exx);
+  __syncthreads();   // sm.sc
   {
-    // one power-of-two normalisation of the X operand for the whole head, from
-    // the largest column scale (COL) and the largest |k| of the period
-    float smax = 0.f, kmax = 0.f;
-    for (int j = lane; j < D; j += 32) smax = fmaxf(smax, __half2float(__ushort_as_half(s_sc[j])));
-    constexpr int EPW = 16 / C::ESZ;                       // elements per 16-byte load
-    for (int i = lane; i < P * D / EPW; i += 32) {
-      const int s2 = i / (D / EPW), jv = i - s2 * (D / EPW);
-      const uint4 v4 = *reinterpret_cast<const uint4*>(s_kv + (size_t)(s2 * 2 * D + jv * EPW) * C::ESZ);
-      const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+    // X operand, built by fragment owner: entry (x, ks, g, t) holds rows
+    // k = 2t, 2t+1 | 2t+8, 2t+9 (key channels jof(t, ks, 0..3)) of column
+    // 8x + g = vector s = 4x + g/2, hi (g even) or lo (g odd) part.  One item
+    // writes the hi and the lo entry of one (x, ks, g/2, t).
+    for (int it = tid; it < NTX * KS * 16; it += C::THREADS) {
+      const int tt = it & 3, gp = (it >> 2) & 3, xk = it >> 4;   // xk = x * KS + ks
+      const int ks = xk % KS, x = xk / KS;
+      const int s = 4 * x + gp;
+      uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+      if (s < P) {
+        __half hv[4], lv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (BF16) {
-          kmax = fmaxf(kmax, __uint_as_float((wv[e] << 16) & 0x7fffffffu));
-          kmax = fmaxf(kmax, __uint_as_float(wv[e] & 0x7fff0000u));
-        } else {
-          kmax = fmaxf(kmax, __uint_as_float(wv[e] & 0x7fffffffu));
+        for (int pos = 0; pos < 4; ++pos) {
+          const int j = jof<D, BITS>(tt, ks, pos);
+          const float kv = io_at(s_kv, s * 2 * D + j, BF16);
+          const float xv = (col ? kv * sm.sc[j] : kv) * upx;
+          hv[pos] = __float2half_rn(xv);
+          lv[pos] = __float2half_rn(xv - __half2float(hv[pos]));
         }
+        hw[0] = h2u(__halves2half2(hv[0], hv[1]));
+        hw[1] = h2u(__halves2half2(hv[2], hv[3]));
+        lw[0] = h2u(__halves2half2(lv[0], lv[1]));
+        lw[1] = h2u(__halves2half2(lv[2], lv[3]));
       }
+      sm.bx[x][ks][2 * gp][tt] = make_uint2(hw[0], hw[1]);
+      sm.bx[x][ks][2 * gp + 1][tt] = make_uint2(lw[0], lw[1]);
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      smax = fmaxf(smax, __shfl_xor_sync(FULL, smax, off));
-      kmax = fmaxf(kmax, __shfl_xor_sync(FULL, kmax, off));
-    }
-    const float bmax = col ? smax * kmax : kmax;
-    int exx = 0;
-    if (bmax >= 1.17549435e-38f && bmax < INFINITY) exx = max(-120, min(120, 14 - exp2_floor(bmax)));
-    const float upx = pow2i(exx);
-    if (tid == 0) sm.xinv = pow2i(-exx);
-    // X operand: element (s, j) -> hi / lo f16 at its fragment position in
-    // columns 2s / 2s+1 (8 columns per tile)
-    __half* bxh = reinterpret_cast<__half*>(&sm.bx[0][0][0][0]);
-    for (int idx = tid; idx < P * D; idx += C::THREADS) {
-      const int s = idx / D, j = idx - (idx / D) * D;
-      const float kv = io_at(s_kv, s * 2 * D + j, BF16);
-      const float x = (col ? kv * __half2float(__ushort_as_half(s_sc[j])) : kv) * upx;
-      const __half hi = __float2half_rn(x);
-      const __half lo = __float2half_rn(x - __half2float(hi));
-      int tt, ks, pos;
-      kslot_of<D, BITS>(j, tt, ks, pos);
-      const int c0 = 2 * s, tile = c0 >> 3, gc = c0 & 7;
-      const size_t at = ((((size_t)tile * KS + ks) * 8 + gc) * 4 + tt) * 4 + pos;
-      bxh[at] = hi;
-      bxh[at + 16] = lo;                         // column gc + 1 of the same tile
-    }
-    // update B: column n = g of tile 2ks + hs is key channel jof(g>>1, ks, 2hs + (g&1));
-    // k-step u, lane group t holds slots 16u + 2t + {0, 1} (b0) and + {8, 9} (b1);
-    // slot sigma is token sigma % PMAX of segment sigma / PMAX (K, K, K_lo)
-    for (int cix = tid; cix < NT * 8; cix += C::THREADS) {
-      const int tau = cix >> 3, gg = cix & 7;
+    // update B, built by fragment owner: entry (tau, u, g, t): column n = g of
+    // tile tau = 2ks + hs is key channel jof(g/2, ks, 2hs + g%2); rows are the
+    // k-slots 16u + 2t + {0, 1} (b0) and + {8, 9} (b1); slot sigma is token
+    // sigma % PMAX of segment sigma / PMAX (K, K, K_lo)
+    for (int it = tid; it < NT * KU * 32; it += C::THREADS) {
+      const int tt = it & 3, gg = (it >> 2) & 7, tu = it >> 5;   // tu = tau * KU + u
+      const int u = tu % KU, tau = tu / KU;
       const int j = jof<D, BITS>(gg >> 1, tau >> 1, 2 * (tau & 1) + (gg & 1));
-      __half kh[PMAX], kl[PMAX];
+      uint32_t wv[2];
 #pragma unroll
-      for (int s2 = 0; s2 < PMAX; ++s2) {
-        const float kv = s2 < P ? io_at(s_kv, s2 * 2 * D + j, BF16) : 0.f;
-        kh[s2] = __float2half_rn(kv);
-        kl[s2] = C::NSEG == 3 ? __float2half_rn(kv - __half2float(kh[s2])) : kh[s2];
-      }
+      for (int q2 = 0; q2 < 2; ++q2) {
+        __half hv[2];
 #pragma unroll
-      for (int u = 0; u < KU; ++u)
-#pragma unroll
-        for (int tt = 0; tt < 4; ++tt) {
-          uint32_t wv[2];
-#pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            __half hv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int sigma = 16 * u + 2 * tt + e + 8 * q2;
-              const int seg = sigma / PMAX, s2 = sigma % PMAX;
-              hv[e] = seg >= C::NSEG ? __ushort_as_half((unsigned short)0) : (seg == 2 ? kl[s2] : kh[s2]);
-            }
-            wv[q2] = h2u(__halves2half2(hv[0], hv[1]));
+        for (int e = 0; e < 2; ++e) {
+          const int sigma = 16 * u + 2 * tt + e + 8 * q2;
+          const int seg = sigma / PMAX, s2 = sigma % PMAX;
+          __half h = __ushort_as_half((unsigned short)0);
+          if (seg < C::NSEG && s2 < P) {
+            const float kv = io_at(s_kv, s2 * 2 * D + j, BF16);
+            h = __float2half_rn(kv);
+            if (seg == 2) h = __float2half_rn(kv - __half2float(h));
           }
-          sm.bkf[tau][u][gg][tt] = make_uint2(wv[0], wv[1]);
+          hv[e] = h;
         }
+        wv[q2] = h2u(__halves2half2(hv[0], hv[1]));
+      }
+      sm.bkf[tau][u][gg][tt] = make_uint2(wv[0], wv[1]);
     }
   }
   __syncthreads();
@@ -568,10 +553,6 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
   Smem<D, BF16, PMAX>& sm = *reinterpret_cast<Smem<D, BF16, PMAX>*>(smem_raw);
   const int tid = threadIdx.x;
   const int n_heads = p.B * p.H;
-  {   // operand columns that stay unused (vectors >= P) must read as zero
-    uint32_t* z = reinterpret_cast<uint32_t*>(&sm.bx[0][0][0][0]);
-    for (int i = tid; i < (int)(sizeof(sm.bx) / 4); i += C::THREADS) z[i] = 0u;
-  }
   if (tid == 0) {
     mbar_init(&sm.bar[0], 1);
     mbar_init(&sm.bar[1], 1);

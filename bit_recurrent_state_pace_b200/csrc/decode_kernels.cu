@@ -59,8 +59,8 @@ struct Stage {
   static constexpr int SC = 3 * D * ESZ;                          // fp16 scales [D]
   static constexpr int KV = SC + 2 * D;                           // rows [PMAX-1][k | v]
   static constexpr int AB = KV + (PMAX - 1) * 2 * D * ESZ;        // gates [PMAX][2]
-  static constexpr int G = AB + (2 * PMAX * ESZ + 15) / 16 * 16;  // Gram [PMAX][PMAX] + [PMAX]
-  static constexpr int BYTES = G + (4 * PMAX * (PMAX + 1) + 15) / 16 * 16;
+  static constexpr int G = AB + (2 * PMAX * ESZ + 15) / 16 * 16;  // Gram block
+  static constexpr int BYTES = G + (4 * (PMAX * (PMAX + 1) + 2) + 15) / 16 * 16;
   // two stages (copies one head ahead) while 8 warps fit twice per SM
   static constexpr int N = 2 * 8 * 2 * BYTES <= 160 * 1024 ? 2 : 1;
 };
@@ -398,8 +398,31 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
 
   // 12. period end (n == P): replace the Gram block by the commit's chunk-form
   //     factors W[t][s] = gamma_{P/t} T[t][s] beta_s, T = (I + A)^{-1} (lane s
-  //     solves column s by forward substitution), followed by gamma_s
+  //     solves column s by forward substitution), followed by gamma_s, the
+  //     largest |k| of the period and the largest stored scale
   if (n == P) {
+    float km = 0.f, sm = 0.f;
+    {
+      float x[EPL];
+#pragma unroll
+      for (int s = 0; s < PMAX; ++s) {
+        if (s < n) {
+          load_f<EPL, BF16>(s < n - 1 ? stg + ST::KV : stg + ST::K,
+                            s < n - 1 ? s * row_elems + (size_t)EPL * lane : (size_t)EPL * lane, x);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) km = fmaxf(km, fabsf(x[e]));
+        }
+      }
+      Raw<EPL, true> s_raw;
+      s_raw.load(stg + ST::SC, (size_t)EPL * lane);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) sm = fmaxf(sm, fabsf(s_raw.get_half(e)));
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        km = fmaxf(km, __shfl_xor_sync(FULL, km, off));
+        sm = fmaxf(sm, __shfl_xor_sync(FULL, sm, off));
+      }
+    }
     __syncwarp();
     float Tc[PMAX];
 #pragma unroll
@@ -417,6 +440,10 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
       for (int tt = 0; tt < PMAX; ++tt)
         if (tt < P) gw[tt * P + lane] = scr.gsb[1][tt] * Tc[tt] * bs;
       gw[P * P + lane] = scr.gsb[0][lane];
+    }
+    if (lane == 0) {
+      gw[P * P + P] = km;
+      gw[P * P + P + 1] = sm;
     }
   }
   __syncwarp();

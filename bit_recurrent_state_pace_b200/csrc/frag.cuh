@@ -163,6 +163,11 @@ struct Raw {
       *reinterpret_cast<uint16_t*>(p) = (uint16_t)w[0];
     }
   }
+  // element e read as fp16 (the 16-bit layout shared with bf16)
+  __device__ __forceinline__ float get_half(int e) const {
+    const uint32_t x = w[e >> 1];
+    return __half2float(__ushort_as_half((unsigned short)((e & 1) ? (x >> 16) : (x & 0xffffu))));
+  }
   __device__ __forceinline__ float get(int e) const {
     if (BF16) {
       const uint32_t x = w[e >> 1];

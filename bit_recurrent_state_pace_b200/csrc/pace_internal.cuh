@@ -23,9 +23,9 @@ struct PoolDev {
   uint8_t* state;             // [B][slot_stride]
   uint8_t* kv;                // [B][H][P][d_k + d_v] io elements
   uint8_t* ab;                // [B][H] blocks of ab_stride bytes: [P][2] io elements
-  uint8_t* gram;              // [B][H] blocks of gram_stride bytes: [P][P] + [P] fp32
+  uint8_t* gram;              // [B][H] blocks of gram_stride bytes: [P][P] + [P] + [2] fp32
   uint32_t ab_stride;         // round_up(2 P io bytes, 16)
-  uint32_t gram_stride;       // round_up(4 P (P + 1), 16)
+  uint32_t gram_stride;       // round_up(4 (P (P + 1) + 2), 16)
   int32_t* fill;              // [B][H]
   uint32_t* flags;            // status word
   uint32_t rec_off[PACE_MAX_HEADS];   // record offset of head h inside a slot
@@ -63,7 +63,7 @@ __host__ __device__ inline uint32_t ab_stride_bytes(int P, int io) {
 }
 
 __host__ __device__ inline uint32_t gram_stride_bytes(int P) {
-  return (uint32_t)round_up((size_t)4 * P * (P + 1), 16);
+  return (uint32_t)round_up((size_t)4 * (P * (P + 1) + 2), 16);
 }
 
 // Load element `idx` of an io-dtype array as fp32.

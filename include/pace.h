@@ -89,15 +89,16 @@ typedef struct {
  *          byte offset round_up(size(KV), 256) region AB: [B][H] blocks of
  *          round_up(2*P*io_size, 16) bytes, each [P][2] io_dtype elements
  *          (alpha, beta); then at the next 256-byte boundary region G: [B][H]
- *          blocks of round_up(4*P*(P+1), 16) bytes, each [P][P] + [P] fp32.
- *          While a period fills, G[t][s] = k_t . k_s for s < t, the Gram
- *          entries of the buffered keys, written by the decode step that
- *          buffers token t (so each step computes only its own).  The step
- *          that buffers the P-th token replaces them with the period's
+ *          blocks of round_up(4*(P*(P+1)+2), 16) bytes, each [P][P] + [P]
+ *          + [2] fp32.  While a period fills, G[t][s] = k_t . k_s for s < t,
+ *          the Gram entries of the buffered keys, written by the decode step
+ *          that buffers token t (so each step computes only its own).  The
+ *          step that buffers the P-th token replaces them with the period's
  *          chunk-form factors for the commit: W[s][s'] = gamma_{P/s}
- *          T[s][s'] beta_s' with T = (I + A)^{-1}, and after it the P decay
- *          products gamma_s.  q is not stored: no later step reads an old
- *          query.
+ *          T[s][s'] beta_s' with T = (I + A)^{-1}, then the P decay products
+ *          gamma_s, then max |k_s[j]| over the period's keys and the largest
+ *          stored scale of the head.  q is not stored: no later step reads
+ *          an old query.
  * aux    : fill counters int32 [B][H] (tokens in each head's buffer), then at
  *          byte offset round_up(4*B*H, 256) the uint32 status word.
  * All three regions must be 256-byte aligned.

@@ -45,7 +45,7 @@ def test_pool_byte_accounting():
     st, buf, aux = pace.pace_pool_bytes(4096, 48, 128, 128, 8, 0, 0, bits)
     assert st == 4096 * (12 * 16640 + 36 * 8448) == 2063597568
     # k,v rows; alpha,beta rows (32 B per head); Gram cache (256 B per head)
-    assert buf == 4096 * 48 * 8 * 512 + 4096 * 48 * 32 + 4096 * 48 * 288
+    assert buf == 4096 * 48 * 8 * 512 + 4096 * 48 * 32 + 4096 * 48 * 304
     # mixed 4/8 pool against an all-INT8 pool: 0.631 (the pages' "about two
     # thirds" of 8-bit memory, "PACE: four-bit recurrent state by rounding less
     # often", TL;DR; there the 8-bit baseline also keeps FP16 channels)
