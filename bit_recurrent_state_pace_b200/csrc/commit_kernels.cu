@@ -65,7 +65,10 @@ struct Cfg {
   static constexpr int NU = PMAX >= 16 ? 4 : 2;     // distinct U^ rows a lane feeds
   static constexpr int ESZ = BF16 ? 2 : 4;
   static constexpr int REC = (D * D + 2 * D + 15) / 16 * 16;   // largest record (INT8)
-  static constexpr int KVB = PMAX * 2 * D * ESZ;
+  // buffered rows sit 16 bytes apart from a multiple of 128 so that the same
+  // key channel of different tokens falls in different shared-memory banks
+  static constexpr int ROWS = 2 * D * ESZ + 16;
+  static constexpr int KVB = PMAX * ROWS;
   static constexpr int ABB = (2 * PMAX * ESZ + 15) / 16 * 16;
   static constexpr int GRB = (4 * (PMAX * (PMAX + 1) + 2) + 15) / 16 * 16;
   static constexpr int SLOT = REC + KVB + ABB + GRB;
@@ -113,7 +116,8 @@ __device__ __forceinline__ void issue_head(const PoolDev& p, int head, Smem<D, B
   fence_proxy_async_smem();
   mbar_arrive_expect_tx(&sm.bar[s], rec_bytes + kv_bytes + p.ab_stride + p.gram_stride);
   tma_load_1d(dst, rec, rec_bytes, &sm.bar[s]);
-  tma_load_1d(dst + C::REC, kv, kv_bytes, &sm.bar[s]);
+  for (int r = 0; r < p.P; ++r)
+    tma_load_1d(dst + C::REC + r * C::ROWS, kv + (size_t)r * 2 * D * C::ESZ, 2 * D * C::ESZ, &sm.bar[s]);
   tma_load_1d(dst + C::REC + C::KVB, ab, p.ab_stride, &sm.bar[s]);
   tma_load_1d(dst + C::REC + C::KVB + C::ABB, gr, p.gram_stride, &sm.bar[s]);
 }
@@ -204,8 +208,8 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
     // 8x + g = vector s = 4x + g/2, hi (g even) or lo (g odd) part.  One item
     // writes the hi and the lo entry of one (x, ks, g/2, t).
     for (int it = tid; it < NTX * KS * 16; it += C::THREADS) {
-      const int tt = it & 3, gp = (it >> 2) & 3, xk = it >> 4;   // xk = x * KS + ks
-      const int ks = xk % KS, x = xk / KS;
+      const int tt = it & 3, ks = (it >> 2) % KS, rest = (it >> 2) / KS;
+      const int gp = rest & 3, x = rest >> 2;
       const int s = 4 * x + gp;
       uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
       if (s < P) {
@@ -213,7 +217,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 #pragma unroll
         for (int pos = 0; pos < 4; ++pos) {
           const int j = jof<D, BITS>(tt, ks, pos);
-          const float kv = io_at(s_kv, s * 2 * D + j, BF16);
+          const float kv = io_at(s_kv + s * C::ROWS, j, BF16);
           const float xv = (col ? kv * sm.sc[j] : kv) * upx;
           hv[pos] = __float2half_rn(xv);
           lv[pos] = __float2half_rn(xv - __half2float(hv[pos]));
@@ -223,8 +227,10 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
         lw[0] = h2u(__halves2half2(lv[0], lv[1]));
         lw[1] = h2u(__halves2half2(lv[2], lv[3]));
       }
-      sm.bx[x][ks][2 * gp][tt] = make_uint2(hw[0], hw[1]);
-      sm.bx[x][ks][2 * gp + 1][tt] = make_uint2(lw[0], lw[1]);
+      // stored at row slot g ^ (ks & 3): a permutation inside each 256-byte
+      // [g][t] block that spreads these stores over the banks
+      sm.bx[x][ks][(2 * gp) ^ (ks & 3)][tt] = make_uint2(hw[0], hw[1]);
+      sm.bx[x][ks][(2 * gp + 1) ^ (ks & 3)][tt] = make_uint2(lw[0], lw[1]);
     }
     // update B, built by fragment owner: entry (tau, u, g, t): column n = g of
     // tile tau = 2ks + hs is key channel jof(g/2, ks, 2hs + g%2); rows are the
@@ -244,7 +250,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
           const int seg = sigma / PMAX, s2 = sigma % PMAX;
           __half h = __ushort_as_half((unsigned short)0);
           if (seg < C::NSEG && s2 < P) {
-            const float kv = io_at(s_kv, s2 * 2 * D + j, BF16);
+            const float kv = io_at(s_kv + s2 * C::ROWS, j, BF16);
             h = __float2half_rn(kv);
             if (seg == 2) h = __float2half_rn(kv - __half2float(h));
           }
@@ -274,7 +280,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
     for (int x = 0; x < NTX; ++x) {
-      const uint2 bb = sm.bx[x][ks][g][t];
+      const uint2 bb = sm.bx[x][ks][g ^ (ks & 3)][t];
       mma16816(xacc[x], Af[ks], bb.x, bb.y);
     }
   // r_s = v_s - gamma_s x_s for this lane's vectors s = 4x + t, then all-gather in the quad
@@ -289,8 +295,8 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       ro[x][0] = ro[x][1] = 0.f;
       if (s < P) {
         const float gs = gam[s];
-        ro[x][0] = io_at(s_kv, s * 2 * D + D + i0, BF16) - gs * ((xacc[x][0] + xacc[x][1]) * s0);
-        ro[x][1] = io_at(s_kv, s * 2 * D + D + i1, BF16) - gs * ((xacc[x][2] + xacc[x][3]) * s1);
+        ro[x][0] = io_at(s_kv + s * C::ROWS, D + i0, BF16) - gs * ((xacc[x][0] + xacc[x][1]) * s0);
+        ro[x][1] = io_at(s_kv + s * C::ROWS, D + i1, BF16) - gs * ((xacc[x][2] + xacc[x][3]) * s1);
       }
     }
 #pragma unroll
@@ -312,12 +318,23 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 #pragma unroll
   for (int q = 0; q < NU; ++q) {
     const int s = (2 * t + (q & 1) + 8 * (q >> 1)) % PMAX;
+    float wrow[PMAX];
+    if ((P & 3) == 0 && s < P) {          // row s of W in 16-byte pieces
+#pragma unroll
+      for (int c = 0; c < PMAX / 4; ++c) {
+        const float4 w4 = 4 * c < P ? reinterpret_cast<const float4*>(W + s * P)[c]
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        wrow[4 * c] = w4.x; wrow[4 * c + 1] = w4.y; wrow[4 * c + 2] = w4.z; wrow[4 * c + 3] = w4.w;
+      }
+    } else {
+#pragma unroll
+      for (int sp = 0; sp < PMAX; ++sp) wrow[sp] = (s < P && sp < P) ? W[s * P + sp] : 0.f;
+    }
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int sp = 0; sp < PMAX; ++sp) {
-      const float wv = (s < P && sp < P) ? W[s * P + sp] : 0.f;
-      a0 = fmaf(wv, r[sp][0], a0);
-      a1 = fmaf(wv, r[sp][1], a1);
+      a0 = fmaf(wrow[sp], r[sp][0], a0);
+      a1 = fmaf(wrow[sp], r[sp][1], a1);
     }
     uh[q][0] = a0;
     uh[q][1] = a1;
