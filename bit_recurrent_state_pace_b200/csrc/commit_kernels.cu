@@ -506,15 +506,15 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   const float qr0 = col ? 0.f : (slow ? sm.sfv[i0] : sm.qf[i0] * down);
   const float qr1 = col ? 0.f : (slow ? sm.sfv[i1] : sm.qf[i1] * down);
   auto encode_rows = [&](auto fast) {
-    // magic f16 pair of value (ks_a, pos_a) and (ks_b, pos_b) of row half rr;
-    // value (ks, pos) sits in tile 2ks + (pos >> 1), element pos & 1
-    auto mk = [&](int ksa, int pa, int ksb, int pb, int rr) -> uint32_t {
-      const float a = acc[2 * ksa + (pa >> 1)][2 * rr + (pa & 1)];
-      const float bq = acc[2 * ksb + (pb >> 1)][2 * rr + (pb & 1)];
+    // magic f16 pair of tile tau, row half rr: elements (2rr, 2rr + 1) are the
+    // key channels jof(t, tau / 2, 2 (tau % 2) + {0, 1}), adjacent registers
+    auto hq = [&](int tau, int rr) -> uint32_t {
+      const float a = acc[tau][2 * rr], bq = acc[tau][2 * rr + 1];
       float qa = rr ? qr1 : qr0, qb = qa;
       if (col) {
-        qa = pick4(wt.q[ksa][t], pa);
-        qb = pick4(wt.q[ksb][t], pb);
+        const float4 q4 = wt.q[tau >> 1][t];
+        qa = (tau & 1) ? q4.z : q4.x;
+        qb = (tau & 1) ? q4.w : q4.y;
       }
       if (decltype(fast)::value) return magic_fast<BITS>(a, bq, qa, qb);
       return magic_exact<BITS>(a * down, bq * down, qa, qb);
@@ -523,15 +523,17 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
     for (int rr = 0; rr < 2; ++rr) {
       uint8_t* row = rec + (size_t)(rr ? i1 : i0) * ROWB;
       if (BITS == 4) {
-        // word m holds channels 8m + k of the lane's range: k-step 2m gives
-        // k = 0 (pos 0), 4 (pos 1), 1 (pos 2), 5 (pos 3); k-step 2m+1 gives k + 2
+        // word m holds channels 8m + k of the lane's range; tiles 4m .. 4m+3
+        // hold k = (0, 4), (1, 5), (2, 6), (3, 7), each code in the low byte
+        // of its f16 half
         constexpr int NW = D / 32;
         uint32_t wd[NW];
 #pragma unroll
         for (int m = 0; m < NW; ++m) {
-          const int ka = 2 * m, kb = 2 * m + 1;
-          const uint32_t E = prmt(mk(ka, 0, kb, 0, rr), mk(ka, 1, kb, 1, rr), 0x6420u);  // k 0 2 4 6
-          const uint32_t O = prmt(mk(ka, 2, kb, 2, rr), mk(ka, 3, kb, 3, rr), 0x6420u);  // k 1 3 5 7
+          const uint32_t h04 = hq(4 * m, rr), h15 = hq(4 * m + 1, rr);
+          const uint32_t h26 = hq(4 * m + 2, rr), h37 = hq(4 * m + 3, rr);
+          const uint32_t E = prmt(h04, h26, 0x6240u);   // k 0 2 4 6
+          const uint32_t O = prmt(h15, h37, 0x6240u);   // k 1 3 5 7
           wd[m] = (E | (O << 4)) ^ 0x88888888u;
         }
         uint8_t* dst = row + chunk_offset<D, 4>(t, 0);
@@ -539,7 +541,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
         else if (NW == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[1]);
         else *reinterpret_cast<uint32_t*>(dst) = wd[0];
       } else {
-        // k-step ks covers channels base + pos of one code word
+        // k-step ks covers channels base + pos of one code word: tiles 2ks, 2ks+1
         constexpr int WPC = D / 32;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -547,7 +549,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 #pragma unroll
           for (int m = 0; m < WPC; ++m) {
             const int ks = c * WPC + m;
-            wd[m] = prmt(mk(ks, 0, ks, 1, rr), mk(ks, 2, ks, 3, rr), 0x6420u) ^ 0x80808080u;
+            wd[m] = prmt(hq(2 * ks, rr), hq(2 * ks + 1, rr), 0x6420u) ^ 0x80808080u;
           }
           uint8_t* dst = row + chunk_offset<D, 8>(t, c);
           if (WPC == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
