@@ -171,13 +171,15 @@ __device__ __forceinline__ float pick4(const float4& f, int i) {
   return i == 0 ? f.x : i == 1 ? f.y : i == 2 ? f.z : f.w;
 }
 
-template <int D, bool BF16, int PMAX, int BITS>
+// EXACT: the pool's period equals PMAX, so every loop bound over tokens is a
+// compile-time constant.
+template <int D, bool BF16, int PMAX, int BITS, bool EXACT>
 __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot) {
   using C = Cfg<D, BF16, PMAX>;
   constexpr int KS = C::KS, NT = C::NT, NTX = C::NTX, KU = C::KU, NU = C::NU;
   constexpr int ROWB = D * BITS / 8;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
-  const int P = p.P, h = head % p.H, b = head / p.H;
+  const int P = EXACT ? PMAX : p.P, h = head % p.H, b = head / p.H;
   const bool col = p.axis == PACE_SCALE_COL;
   const int qmax = BITS == 4 ? 7 : 127;
   uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
@@ -564,7 +566,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   if (tid == 0) p.fill[head] = 0;
 }
 
-template <int D, bool BF16, int PMAX>
+template <int D, bool BF16, int PMAX, bool EXACT>
 __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     commit_kernel(PoolDev p) {
   using C = Cfg<D, BF16, PMAX>;
@@ -572,6 +574,9 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
   Smem<D, BF16, PMAX>& sm = *reinterpret_cast<Smem<D, BF16, PMAX>*>(smem_raw);
   const int tid = threadIdx.x;
   const int n_heads = p.B * p.H;
+  // thread 0 keeps the candidate after the next head and its fill count,
+  // loaded one head ahead so that the load's latency is hidden
+  int cand = n_heads, cand_fill = 0;
   if (tid == 0) {
     mbar_init(&sm.bar[0], 1);
     mbar_init(&sm.bar[1], 1);
@@ -580,6 +585,8 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     const int first = find_full(p, blockIdx.x, gridDim.x, n_heads);
     sm.next_head = first;
     if (first < n_heads) issue_head<D, BF16, PMAX>(p, first, sm, 0);
+    cand = first + gridDim.x;
+    if (cand < n_heads) cand_fill = p.fill[cand];
   }
   __syncthreads();
   uint32_t parity[2] = {0u, 0u};
@@ -588,9 +595,12 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
   while (head < n_heads) {
     __syncthreads();                      // everyone has read next_head; slot s^1 is free
     if (tid == 0) {
-      const int nxt = find_full(p, head + gridDim.x, gridDim.x, n_heads);
+      int nxt = cand;
+      if (nxt < n_heads && cand_fill != p.P) nxt = find_full(p, nxt + gridDim.x, gridDim.x, n_heads);
       sm.next_head = nxt;
       if (nxt < n_heads) issue_head<D, BF16, PMAX>(p, nxt, sm, s ^ 1);
+      cand = nxt + gridDim.x;
+      if (cand < n_heads) cand_fill = p.fill[cand];
     }
     const bool ok = mbar_wait_bounded(&sm.bar[s], parity[s], p.flags);
     parity[s] ^= 1u;
@@ -602,9 +612,9 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
       return;
     }
     if (p.bits[head % p.H] == 4)
-      commit_head<D, BF16, PMAX, 4>(p, head, sm, sm.slot[s]);
+      commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s]);
     else
-      commit_head<D, BF16, PMAX, 8>(p, head, sm, sm.slot[s]);
+      commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s]);
     __syncthreads();
     if (tid == 0) sm.slow = 0;
     head = sm.next_head;
@@ -625,25 +635,30 @@ int sm_count_dev() {
   return cached[dev];
 }
 
-template <int D, bool BF16, int PMAX>
+template <int D, bool BF16, int PMAX, bool EXACT>
 cudaError_t launch_t(const PoolDev& p, cudaStream_t st) {
   using C = Cfg<D, BF16, PMAX>;
   const size_t smem = sizeof(Smem<D, BF16, PMAX>);
-  cudaError_t e = cudaFuncSetAttribute(commit_kernel<D, BF16, PMAX>,
+  cudaError_t e = cudaFuncSetAttribute(commit_kernel<D, BF16, PMAX, EXACT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long heads = (long)p.B * p.H;
   long blocks = 2L * sm_count_dev() * (D == 128 ? 1 : D == 64 ? 2 : 4);
   if (blocks > heads) blocks = heads;
-  commit_kernel<D, BF16, PMAX><<<(unsigned)blocks, C::THREADS, smem, st>>>(p);
+  commit_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, C::THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 template <int D, bool BF16>
 cudaError_t launch_p(const PoolDev& p, cudaStream_t st) {
-  if (p.P <= 4) return launch_t<D, BF16, 4>(p, st);
-  if (p.P <= 8) return launch_t<D, BF16, 8>(p, st);
-  return launch_t<D, BF16, 16>(p, st);
+  switch (p.P) {
+    case 4: return launch_t<D, BF16, 4, true>(p, st);
+    case 8: return launch_t<D, BF16, 8, true>(p, st);
+    case 16: return launch_t<D, BF16, 16, true>(p, st);
+  }
+  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, st);
+  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, st);
+  return launch_t<D, BF16, 16, false>(p, st);
 }
 
 }  // namespace

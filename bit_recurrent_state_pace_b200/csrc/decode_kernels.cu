@@ -85,7 +85,8 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
   return r;
 }
 
-template <int D, bool BF16, int PMAX, int BITS>
+// EXACT: the pool's period equals PMAX (compile-time loop bounds over tokens).
+template <int D, bool BF16, int PMAX, int BITS, bool EXACT>
 __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, const void* __restrict__ q,
                                             const void* __restrict__ k, const void* __restrict__ v,
                                             const void* __restrict__ alpha,
@@ -96,7 +97,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   constexpr int ESZ = BF16 ? 2 : 4;
   const int g = lane >> 2, t = lane & 3;
   const int h = head % p.H, b = head / p.H;
-  const int P = p.P;
+  const int P = EXACT ? PMAX : p.P;
   const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
 
   // 1. start streaming the first row blocks of codes
@@ -477,7 +478,7 @@ __device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill
   }
 }
 
-template <int D, bool BF16, int PMAX>
+template <int D, bool BF16, int PMAX, bool EXACT>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_step_kernel(PoolDev p, const void* __restrict__ q, const void* __restrict__ k,
                        const void* __restrict__ v, const void* __restrict__ alpha,
@@ -549,9 +550,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int n = nprev + 1;
     if (p.bits[head % p.H] == 4)
-      decode_head<D, BF16, PMAX, 4>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
+      decode_head<D, BF16, PMAX, 4, EXACT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
     else
-      decode_head<D, BF16, PMAX, 8>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
+      decode_head<D, BF16, PMAX, 8, EXACT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
   }
 }
 
@@ -568,29 +569,34 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, bool BF16, int PMAX>
+template <int D, bool BF16, int PMAX, bool EXACT>
 cudaError_t launch_t(const PoolDev& p, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
   using ST = Stage<D, BF16, PMAX>;
   const size_t smem = (size_t)kWarpsPerBlock * (ST::N * ST::BYTES + sizeof(WarpScratch<D>) +
                                                 ST::N * sizeof(uint64_t));
-  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX>,
+  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX, EXACT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long heads = (long)p.B * p.H;
   long blocks = (heads + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const long cap = 2L * sm_count();
   if (blocks > cap) blocks = cap;
-  decode_step_kernel<D, BF16, PMAX><<<(unsigned)blocks, kThreads, smem, st>>>(p, q, k, v, alpha, beta, o);
+  decode_step_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, kThreads, smem, st>>>(p, q, k, v, alpha, beta, o);
   return cudaGetLastError();
 }
 
 template <int D, bool BF16>
 cudaError_t launch_p(const PoolDev& p, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
-  if (p.P <= 4) return launch_t<D, BF16, 4>(p, q, k, v, alpha, beta, o, st);
-  if (p.P <= 8) return launch_t<D, BF16, 8>(p, q, k, v, alpha, beta, o, st);
-  return launch_t<D, BF16, 16>(p, q, k, v, alpha, beta, o, st);
+  switch (p.P) {
+    case 4: return launch_t<D, BF16, 4, true>(p, q, k, v, alpha, beta, o, st);
+    case 8: return launch_t<D, BF16, 8, true>(p, q, k, v, alpha, beta, o, st);
+    case 16: return launch_t<D, BF16, 16, true>(p, q, k, v, alpha, beta, o, st);
+  }
+  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, q, k, v, alpha, beta, o, st);
+  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, q, k, v, alpha, beta, o, st);
+  return launch_t<D, BF16, 16, false>(p, q, k, v, alpha, beta, o, st);
 }
 
 }  // namespace
