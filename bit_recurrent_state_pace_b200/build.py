@@ -40,20 +40,36 @@ def needs_build() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def _run(cmd):
+    return subprocess.run(cmd, capture_output=True, text=True)
+
+
 def build(verbose_ptxas: bool = False, force: bool = False) -> str:
+    """Compile every csrc/*.cu to an object in parallel, then link libpace.so."""
     if not force and not needs_build():
         return LIB
-    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
-           "-Xcompiler", "-fPIC,-O2", "-I", os.path.join(ROOT, "include"),
-           "-o", LIB + ".tmp", *sources()]
+    from concurrent.futures import ThreadPoolExecutor
+    nvcc = nvcc_path()
+    objdir = os.path.join(HERE, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
+             "-I", os.path.join(ROOT, "include")]
     if verbose_ptxas:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    proc = subprocess.run(cmd, capture_output=True, text=True)
+        flags = ["-Xptxas", "-v", *flags]
+    srcs = sources()
+    objs = [os.path.join(objdir, os.path.basename(f)[:-3] + ".o") for f in srcs]
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        procs = list(ex.map(_run, [[nvcc, *flags, "-c", f, "-o", o] for f, o in zip(srcs, objs)]))
+    for proc in procs:
+        if proc.returncode != 0:
+            sys.stderr.write(proc.stdout + proc.stderr)
+            raise RuntimeError("nvcc failed building libpace.so")
+        if verbose_ptxas:
+            sys.stderr.write(proc.stderr)
+    proc = _run([nvcc, *ARCH, "-shared", "-o", LIB + ".tmp", *objs])
     if proc.returncode != 0:
         sys.stderr.write(proc.stdout + proc.stderr)
-        raise RuntimeError("nvcc failed building libpace.so")
-    if verbose_ptxas:
-        sys.stderr.write(proc.stderr)
+        raise RuntimeError("linking libpace.so failed")
     os.replace(LIB + ".tmp", LIB)
     return LIB
 
