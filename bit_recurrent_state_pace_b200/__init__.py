@@ -23,6 +23,7 @@ __all__ = [
     "PACE_FLAG_NONFINITE", "PACE_FLAG_SCALE_OVERFLOW", "PACE_FLAG_BUFFER_FULL", "PACE_FLAG_TIMEOUT",
     "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
     "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
+    "pace_decode_step_range", "pace_commit_period_range",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -69,6 +70,8 @@ def _load():
         "pace_pool_export": [P, F32p, P],
         "pace_decode_step": [P, P, P, P, P, P, F32p, P],
         "pace_commit_period": [P, P],
+        "pace_decode_step_range": [P, I32, I32, I32, P, P, P, P, P, F32p, P],
+        "pace_commit_period_range": [P, I32, I32, I32, P],
         "pace_quantize": [F32p, I64, I32, I32, I32, I32, P, U16p, U32p, P],
         "pace_dequantize": [P, U16p, I64, I32, I32, I32, I32, F32p, P],
         "pace_pool_status": [P, P, ctypes.POINTER(ctypes.c_uint32)],
@@ -171,6 +174,19 @@ def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
 
 def pace_commit_period(handle: int, stream=None) -> None:
     _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_decode_step_range(handle: int, slot_begin: int, slot_count: int, blocks_per_sm: int,
+                           q, k, v, alpha, beta, o, stream=None) -> None:
+    _check("pace_decode_step_range",
+           lib.pace_decode_step_range(handle, slot_begin, slot_count, blocks_per_sm, _ptr(q), _ptr(k),
+                                      _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)))
+
+
+def pace_commit_period_range(handle: int, slot_begin: int, slot_count: int, blocks_per_sm: int,
+                             stream=None) -> None:
+    _check("pace_commit_period_range",
+           lib.pace_commit_period_range(handle, slot_begin, slot_count, blocks_per_sm, _stream(stream)))
 
 
 def pace_quantize(S, n_mats, d_k, d_v, bits, axis, codes, scales, flags=None, stream=None) -> None:
@@ -276,6 +292,15 @@ class PacePool:
 
     def commit_period(self, stream=None) -> None:
         pace_commit_period(self.handle, stream)
+
+    def decode_step_range(self, slot_begin, slot_count, q, k, v, alpha, beta, o, blocks_per_sm=0,
+                          stream=None) -> torch.Tensor:
+        pace_decode_step_range(self.handle, slot_begin, slot_count, blocks_per_sm, q, k, v, alpha,
+                               beta, o, stream)
+        return o
+
+    def commit_period_range(self, slot_begin, slot_count, blocks_per_sm=0, stream=None) -> None:
+        pace_commit_period_range(self.handle, slot_begin, slot_count, blocks_per_sm, stream)
 
     def status(self, stream=None) -> int:
         return pace_pool_status(self.handle, stream)

@@ -96,9 +96,10 @@ struct alignas(16) Smem {
   int slow;
 };
 
-__device__ __forceinline__ int find_full(const PoolDev& p, int from, int step, int n_heads) {
+// First head index >= from (stepping by step, below end) with a full buffer.
+__device__ __forceinline__ int find_full(const PoolDev& p, int from, int step, int end) {
   int hd = from;
-  while (hd < n_heads && p.fill[hd] != p.P) hd += step;
+  while (hd < end && p.fill[hd] != p.P) hd += step;
   return hd;
 }
 
@@ -568,12 +569,14 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 
 template <int D, bool BF16, int PMAX, bool EXACT>
 __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
-    commit_kernel(PoolDev p) {
+    commit_kernel(PoolDev p, Span sp) {
   using C = Cfg<D, BF16, PMAX>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem<D, BF16, PMAX>& sm = *reinterpret_cast<Smem<D, BF16, PMAX>*>(smem_raw);
   const int tid = threadIdx.x;
-  const int n_heads = p.B * p.H;
+  // heads [b0 H, (b0 + nb) H) of this launch; n_heads is the end index
+  const int first_head = sp.b0 * p.H;
+  const int n_heads = (sp.b0 + sp.nb) * p.H;
   // thread 0 keeps the candidate after the next head and its fill count,
   // loaded one head ahead so that the load's latency is hidden
   int cand = n_heads, cand_fill = 0;
@@ -582,7 +585,7 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     mbar_init(&sm.bar[1], 1);
     fence_mbar_init();
     sm.slow = 0;
-    const int first = find_full(p, blockIdx.x, gridDim.x, n_heads);
+    const int first = find_full(p, first_head + blockIdx.x, gridDim.x, n_heads);
     sm.next_head = first;
     if (first < n_heads) issue_head<D, BF16, PMAX>(p, first, sm, 0);
     cand = first + gridDim.x;
@@ -636,39 +639,41 @@ int sm_count_dev() {
 }
 
 template <int D, bool BF16, int PMAX, bool EXACT>
-cudaError_t launch_t(const PoolDev& p, cudaStream_t st) {
+cudaError_t launch_t(const PoolDev& p, const Span& sp, cudaStream_t st) {
   using C = Cfg<D, BF16, PMAX>;
   const size_t smem = sizeof(Smem<D, BF16, PMAX>);
   cudaError_t e = cudaFuncSetAttribute(commit_kernel<D, BF16, PMAX, EXACT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long heads = (long)p.B * p.H;
-  long blocks = 2L * sm_count_dev() * (D == 128 ? 1 : D == 64 ? 2 : 4);
+  const long heads = (long)sp.nb * p.H;
+  if (heads == 0) return cudaSuccess;
+  long blocks = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 2) * sm_count_dev() *
+                (D == 128 ? 1 : D == 64 ? 2 : 4);
   if (blocks > heads) blocks = heads;
-  commit_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, C::THREADS, smem, st>>>(p);
+  commit_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, C::THREADS, smem, st>>>(p, sp);
   return cudaGetLastError();
 }
 
 template <int D, bool BF16>
-cudaError_t launch_p(const PoolDev& p, cudaStream_t st) {
+cudaError_t launch_p(const PoolDev& p, const Span& sp, cudaStream_t st) {
   switch (p.P) {
-    case 4: return launch_t<D, BF16, 4, true>(p, st);
-    case 8: return launch_t<D, BF16, 8, true>(p, st);
-    case 16: return launch_t<D, BF16, 16, true>(p, st);
+    case 4: return launch_t<D, BF16, 4, true>(p, sp, st);
+    case 8: return launch_t<D, BF16, 8, true>(p, sp, st);
+    case 16: return launch_t<D, BF16, 16, true>(p, sp, st);
   }
-  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, st);
-  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, st);
-  return launch_t<D, BF16, 16, false>(p, st);
+  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, sp, st);
+  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, sp, st);
+  return launch_t<D, BF16, 16, false>(p, sp, st);
 }
 
 }  // namespace
 
-cudaError_t launch_commit(const PoolDev& p, cudaStream_t st) {
+cudaError_t launch_commit(const PoolDev& p, const Span& sp, cudaStream_t st) {
   const bool bf = p.io == PACE_IO_BF16;
   switch (p.d_k) {
-    case 32: return bf ? launch_p<32, true>(p, st) : launch_p<32, false>(p, st);
-    case 64: return bf ? launch_p<64, true>(p, st) : launch_p<64, false>(p, st);
-    case 128: return bf ? launch_p<128, true>(p, st) : launch_p<128, false>(p, st);
+    case 32: return bf ? launch_p<32, true>(p, sp, st) : launch_p<32, false>(p, sp, st);
+    case 64: return bf ? launch_p<64, true>(p, sp, st) : launch_p<64, false>(p, sp, st);
+    case 128: return bf ? launch_p<128, true>(p, sp, st) : launch_p<128, false>(p, sp, st);
   }
   return cudaErrorInvalidValue;
 }

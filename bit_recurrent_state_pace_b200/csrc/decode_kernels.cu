@@ -482,7 +482,7 @@ template <int D, bool BF16, int PMAX, bool EXACT>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_step_kernel(PoolDev p, const void* __restrict__ q, const void* __restrict__ k,
                        const void* __restrict__ v, const void* __restrict__ alpha,
-                       const void* __restrict__ beta, float* __restrict__ o) {
+                       const void* __restrict__ beta, float* __restrict__ o, Span sp) {
   using ST = Stage<D, BF16, PMAX>;
   constexpr int NS = ST::N;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES +
                                               kWarpsPerBlock * sizeof(WarpScratch<D>)) + NS * wib;
   for (int i = lane; i < D; i += 32) scr.dig[3][i] = 0;
-  const int n_heads = p.B * p.H;
+  const int n_heads = sp.nb * p.H;   // work items of this launch
   const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
   const int W = gridDim.x * kWarpsPerBlock;
   // lane 0 keeps the fill counts of the current head and the next one
@@ -502,26 +502,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = 0; i < NS; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
     if (warp0 < n_heads) {
-      const int h0 = head_in_order(p, warp0);
+      const int h0 = head_in_order(p, warp0, sp.b0, sp.nb);
       f_cur = p.fill[h0];
       if (NS == 2) issue_stage<D, BF16, PMAX>(p, h0, f_cur, q, k, v, stages, &bar[0]);
-      f_nxt = warp0 + W < n_heads ? p.fill[head_in_order(p, warp0 + W)] : 0;
+      f_nxt = warp0 + W < n_heads ? p.fill[head_in_order(p, warp0 + W, sp.b0, sp.nb)] : 0;
     }
   }
   __syncwarp();
   uint32_t parity = 0u;   // bit i: phase of stage i to wait for
   int s = 0;
   for (int it = warp0; it < n_heads; it += W) {
-    const int head = head_in_order(p, it);
-    const int nh = it + W < n_heads ? head_in_order(p, it + W) : n_heads;
+    const int head = head_in_order(p, it, sp.b0, sp.nb);
+    const int nh = it + W < n_heads ? head_in_order(p, it + W, sp.b0, sp.nb) : -1;
     if (lane == 0) {
       if (NS == 2) {
-        if (nh < n_heads)
+        if (nh >= 0)
           issue_stage<D, BF16, PMAX>(p, nh, f_nxt, q, k, v, stages + (s ^ 1) * ST::BYTES, &bar[s ^ 1]);
       } else {
         issue_stage<D, BF16, PMAX>(p, head, f_cur, q, k, v, stages, &bar[0]);
       }
-      if (nh < n_heads) {   // the next head's codes on their way into L2
+      if (nh >= 0) {   // the next head's codes on their way into L2
         const int hh = nh % p.H;
         prefetch_l2(p.state + (size_t)(nh / p.H) * p.slot_stride + p.rec_off[hh],
                     (uint32_t)record_bytes(D, D, p.bits[hh], D));
@@ -530,14 +530,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int nprev = __shfl_sync(FULL, f_cur, 0);
     if (lane == 0) {
       f_cur = f_nxt;
-      f_nxt = it + 2 * W < n_heads ? p.fill[head_in_order(p, it + 2 * W)] : 0;
+      f_nxt = it + 2 * W < n_heads ? p.fill[head_in_order(p, it + 2 * W, sp.b0, sp.nb)] : 0;
     }
     const bool ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, lane == 0 ? p.flags : nullptr);
     parity ^= 1u << s;
     if (!__all_sync(FULL, ok)) {
       // a copy did not land in time: let the other stage's copy finish (bounded)
       // before this warp stops using its shared memory
-      if (NS == 2 && nh < n_heads) mbar_wait_bounded(&bar[s ^ 1], (parity >> (s ^ 1)) & 1u, nullptr);
+      if (NS == 2 && nh >= 0) mbar_wait_bounded(&bar[s ^ 1], (parity >> (s ^ 1)) & 1u, nullptr);
       return;
     }
     const uint8_t* stg = stages + s * ST::BYTES;
@@ -570,7 +570,7 @@ int sm_count() {
 }
 
 template <int D, bool BF16, int PMAX, bool EXACT>
-cudaError_t launch_t(const PoolDev& p, const void* q, const void* k, const void* v,
+cudaError_t launch_t(const PoolDev& p, const Span& sp, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
   using ST = Stage<D, BF16, PMAX>;
   const size_t smem = (size_t)kWarpsPerBlock * (ST::N * ST::BYTES + sizeof(WarpScratch<D>) +
@@ -578,39 +578,42 @@ cudaError_t launch_t(const PoolDev& p, const void* q, const void* k, const void*
   cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX, EXACT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long heads = (long)p.B * p.H;
+  const long heads = (long)sp.nb * p.H;
+  if (heads == 0) return cudaSuccess;
   long blocks = (heads + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  const long cap = 2L * sm_count();
+  const long cap = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 2) * sm_count();
   if (blocks > cap) blocks = cap;
-  decode_step_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, kThreads, smem, st>>>(p, q, k, v, alpha, beta, o);
+  decode_step_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, kThreads, smem, st>>>(p, q, k, v, alpha,
+                                                                                     beta, o, sp);
   return cudaGetLastError();
 }
 
 template <int D, bool BF16>
-cudaError_t launch_p(const PoolDev& p, const void* q, const void* k, const void* v,
+cudaError_t launch_p(const PoolDev& p, const Span& sp, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
   switch (p.P) {
-    case 4: return launch_t<D, BF16, 4, true>(p, q, k, v, alpha, beta, o, st);
-    case 8: return launch_t<D, BF16, 8, true>(p, q, k, v, alpha, beta, o, st);
-    case 16: return launch_t<D, BF16, 16, true>(p, q, k, v, alpha, beta, o, st);
+    case 4: return launch_t<D, BF16, 4, true>(p, sp, q, k, v, alpha, beta, o, st);
+    case 8: return launch_t<D, BF16, 8, true>(p, sp, q, k, v, alpha, beta, o, st);
+    case 16: return launch_t<D, BF16, 16, true>(p, sp, q, k, v, alpha, beta, o, st);
   }
-  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, q, k, v, alpha, beta, o, st);
-  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, q, k, v, alpha, beta, o, st);
-  return launch_t<D, BF16, 16, false>(p, q, k, v, alpha, beta, o, st);
+  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, sp, q, k, v, alpha, beta, o, st);
+  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, sp, q, k, v, alpha, beta, o, st);
+  return launch_t<D, BF16, 16, false>(p, sp, q, k, v, alpha, beta, o, st);
 }
 
 }  // namespace
 
-cudaError_t launch_decode_step(const PoolDev& p, const void* q, const void* k, const void* v,
-                               const void* alpha, const void* beta, float* o, cudaStream_t st) {
+cudaError_t launch_decode_step(const PoolDev& p, const Span& sp, const void* q, const void* k,
+                               const void* v, const void* alpha, const void* beta, float* o,
+                               cudaStream_t st) {
   const bool bf = p.io == PACE_IO_BF16;
   switch (p.d_k) {
-    case 32: return bf ? launch_p<32, true>(p, q, k, v, alpha, beta, o, st)
-                       : launch_p<32, false>(p, q, k, v, alpha, beta, o, st);
-    case 64: return bf ? launch_p<64, true>(p, q, k, v, alpha, beta, o, st)
-                       : launch_p<64, false>(p, q, k, v, alpha, beta, o, st);
-    case 128: return bf ? launch_p<128, true>(p, q, k, v, alpha, beta, o, st)
-                        : launch_p<128, false>(p, q, k, v, alpha, beta, o, st);
+    case 32: return bf ? launch_p<32, true>(p, sp, q, k, v, alpha, beta, o, st)
+                       : launch_p<32, false>(p, sp, q, k, v, alpha, beta, o, st);
+    case 64: return bf ? launch_p<64, true>(p, sp, q, k, v, alpha, beta, o, st)
+                       : launch_p<64, false>(p, sp, q, k, v, alpha, beta, o, st);
+    case 128: return bf ? launch_p<128, true>(p, sp, q, k, v, alpha, beta, o, st)
+                        : launch_p<128, false>(p, sp, q, k, v, alpha, beta, o, st);
   }
   return cudaErrorInvalidValue;
 }

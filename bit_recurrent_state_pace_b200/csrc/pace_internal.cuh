@@ -34,16 +34,24 @@ struct PoolDev {
   int32_t H4;                         // number of 4-bit heads
 };
 
-// The i-th (slot, head) in work order: all 4-bit heads of every slot, then
-// all 8-bit ones, so that the warps of a launch run one code path at a time.
-__device__ __forceinline__ int head_in_order(const PoolDev& p, int i) {
-  const int n4 = p.B * p.H4;
+// The slots a launch works on, and how many blocks per SM it may occupy
+// (fewer than the default leaves room for a launch on another stream).
+struct Span {
+  int32_t b0, nb;            // slots [b0, b0 + nb)
+  int32_t blocks_per_sm;     // 0: the kernel's default
+};
+
+// The i-th (slot, head) of span slots [b0, b0 + nb) in work order: all 4-bit
+// heads of every slot, then all 8-bit ones, so that the warps of a launch run
+// one code path at a time.
+__device__ __forceinline__ int head_in_order(const PoolDev& p, int i, int b0, int nb) {
+  const int n4 = nb * p.H4;
   if (i < n4) {
     const int b = i / p.H4;
-    return b * p.H + p.order[i - b * p.H4];
+    return (b0 + b) * p.H + p.order[i - b * p.H4];
   }
   const int h8 = p.H - p.H4, j = i - n4, b = j / h8;
-  return b * p.H + p.order[p.H4 + j - b * h8];
+  return (b0 + b) * p.H + p.order[p.H4 + j - b * h8];
 }
 
 __host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -90,9 +98,10 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint16_t* scales, int6
                               int d_v, int bits, int axis, float* S, cudaStream_t st);
 cudaError_t launch_pool_load(const PoolDev& p, const float* S, cudaStream_t st);
 cudaError_t launch_pool_export(const PoolDev& p, float* S, cudaStream_t st);
-cudaError_t launch_decode_step(const PoolDev& p, const void* q, const void* k, const void* v,
-                               const void* alpha, const void* beta, float* o, cudaStream_t st);
-cudaError_t launch_commit(const PoolDev& p, cudaStream_t st);
+cudaError_t launch_decode_step(const PoolDev& p, const Span& sp, const void* q, const void* k,
+                               const void* v, const void* alpha, const void* beta, float* o,
+                               cudaStream_t st);
+cudaError_t launch_commit(const PoolDev& p, const Span& sp, cudaStream_t st);
 cudaError_t launch_gdn_step_f32(float* S, const void* q, const void* k, const void* v,
                                 const void* alpha, const void* beta, int io, float* o, int64_t n,
                                 int d_k, int d_v, cudaStream_t st);

@@ -190,17 +190,41 @@ pace_status pace_pool_export(pace_pool* pool, float* S, void* stream) {
   return from_cuda(pace::launch_pool_export(pool->dev, S, as_stream(stream)));
 }
 
-pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, const void* v,
-                             const void* alpha, const void* beta, float* o, void* stream) {
+namespace {
+bool span_ok(const pace_pool* pool, int32_t slot_begin, int32_t slot_count, int32_t blocks_per_sm) {
+  return slot_begin >= 0 && slot_count >= 0 && (int64_t)slot_begin + slot_count <= pool->dev.B &&
+         blocks_per_sm >= 0 && blocks_per_sm <= 8;
+}
+}  // namespace
+
+pace_status pace_decode_step_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
+                                   int32_t blocks_per_sm, const void* q, const void* k,
+                                   const void* v, const void* alpha, const void* beta, float* o,
+                                   void* stream) {
   if (!pool || !q || !k || !v || !alpha || !beta || !o) return PACE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return PACE_ERR_INVALID_ARG;
   if (!aligned(alpha, 4) || !aligned(beta, 4)) return PACE_ERR_INVALID_ARG;
-  return from_cuda(pace::launch_decode_step(pool->dev, q, k, v, alpha, beta, o, as_stream(stream)));
+  if (!span_ok(pool, slot_begin, slot_count, blocks_per_sm)) return PACE_ERR_INVALID_ARG;
+  const pace::Span sp{slot_begin, slot_count, blocks_per_sm};
+  return from_cuda(pace::launch_decode_step(pool->dev, sp, q, k, v, alpha, beta, o, as_stream(stream)));
+}
+
+pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, const void* v,
+                             const void* alpha, const void* beta, float* o, void* stream) {
+  if (!pool) return PACE_ERR_INVALID_ARG;
+  return pace_decode_step_range(pool, 0, pool->dev.B, 0, q, k, v, alpha, beta, o, stream);
+}
+
+pace_status pace_commit_period_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
+                                     int32_t blocks_per_sm, void* stream) {
+  if (!pool || !span_ok(pool, slot_begin, slot_count, blocks_per_sm)) return PACE_ERR_INVALID_ARG;
+  const pace::Span sp{slot_begin, slot_count, blocks_per_sm};
+  return from_cuda(pace::launch_commit(pool->dev, sp, as_stream(stream)));
 }
 
 pace_status pace_commit_period(pace_pool* pool, void* stream) {
   if (!pool) return PACE_ERR_INVALID_ARG;
-  return from_cuda(pace::launch_commit(pool->dev, as_stream(stream)));
+  return pace_commit_period_range(pool, 0, pool->dev.B, 0, stream);
 }
 
 pace_status pace_quantize(const float* S, int64_t n_mats, int32_t d_k, int32_t d_v, int32_t bits,

@@ -162,6 +162,27 @@ pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, cons
 pace_status pace_commit_period(pace_pool* pool, void* stream);
 
 /*
+ * The same two operations restricted to slots [slot_begin, slot_begin +
+ * slot_count) (0 <= slot_begin, slot_begin + slot_count <= num_slots).  q, k,
+ * v, alpha, beta and o keep the full-pool layout; only the rows of the range
+ * are read or written.  blocks_per_sm bounds how many blocks of the launch
+ * each SM may hold (0 = the kernel's default, at most 8): launches on two
+ * streams that each take part of every SM run side by side, which is how
+ * slots at different phases overlap one group's period commit (arithmetic-
+ * bound) with the other slots' decode (memory-bound).  Launches on different
+ * streams must cover disjoint slot ranges.  PACE_ERR_INVALID_ARG for a range
+ * or blocks_per_sm out of bounds.  This scheduling hook has no counterpart on
+ * the pages; it serves continuous batching, where requests start at
+ * different steps.
+ */
+pace_status pace_decode_step_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
+                                   int32_t blocks_per_sm, const void* q, const void* k,
+                                   const void* v, const void* alpha, const void* beta, float* o,
+                                   void* stream);
+pace_status pace_commit_period_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
+                                     int32_t blocks_per_sm, void* stream);
+
+/*
  * Encode n_mats fp32 matrices S [n_mats][d_v][d_k] (device) with one FP16
  * scale per group ([P2] "Channel-Aligned Encoding"):
  *   amax = max|x| (group); s32 = amax/qmax (fp32 divide, round to nearest);
