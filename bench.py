@@ -48,6 +48,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-slots", type=int, default=32)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--schedule", choices=["staggered", "lockstep"], default="lockstep",
+                    help="phases of the slot groups for the headline value (per-kernel numbers "
+                         "always come from a lockstep pass)")
+    ap.add_argument("--stagger-blocks", default="2,2",
+                    help="blocks per SM of the decode and the commit launches in the staggered schedule")
     return ap.parse_args()
 
 
@@ -223,6 +228,58 @@ def workload_config(w, bits):
             "l2": "state pool larger than L2 (no flush needed)", "prefill_tokens": w.warmup}
 
 
+class Staggered:
+    """Continuous-batching phases: the slots form P groups, group g running
+    one token ahead of group g - 1, so that every decode step one group's
+    buffers are full.  Each step the full group is committed and decoded on
+    stream b while the other groups decode on stream a; with both launches
+    held to part of every SM (blocks_per_sm) the commit's arithmetic overlaps
+    the other slots' memory-bound decode.  Over P steps every slot decodes P
+    tokens and commits once, the same work as P lockstep steps + 1 commit."""
+
+    def __init__(self, pace, pool, w, dec_bps: int, com_bps: int):
+        import torch
+        from bit_recurrent_state_pace_b200.ranks import slot_range
+        self.pace, self.pool, self.P = pace, pool, w.P
+        self.groups = [slot_range(w.B, w.P, g) for g in range(w.P)]
+        self.dec_bps, self.com_bps = dec_bps, com_bps
+        self.sa, self.sb = torch.cuda.Stream(), torch.cuda.Stream()
+        self.t = 0
+        self.launches = 0
+
+    def _dec(self, b0, nb, x, o, bps, stream):
+        if nb > 0:
+            self.pace.pace_decode_step_range(self.pool.handle, b0, nb, bps, x["q"], x["k"], x["v"],
+                                             x["alpha"], x["beta"], o, stream.cuda_stream)
+            self.launches += 1
+
+    def preroll(self, toks, outs, stream):
+        """From all fills 0: group g takes g + 1 tokens (group P-1 ends full)."""
+        B = self.groups[-1][0] + self.groups[-1][1]
+        for r in range(self.P):
+            b0 = self.groups[r][0]
+            self._dec(b0, B - b0, toks[r], outs[r], 0, stream)
+        self.t = 1
+
+    def step(self, x, o, main):
+        import torch
+        gf = (-self.t) % self.P
+        b0, nb = self.groups[gf]
+        B = self.groups[-1][0] + self.groups[-1][1]
+        ev = torch.cuda.Event()
+        ev.record(main)
+        self.sa.wait_event(ev)
+        self.sb.wait_event(ev)
+        self.pace.pace_commit_period_range(self.pool.handle, b0, nb, self.com_bps, self.sb.cuda_stream)
+        self.launches += 1
+        self._dec(b0, nb, x, o, self.dec_bps, self.sb)
+        self._dec(0, b0, x, o, self.dec_bps, self.sa)
+        self._dec(b0 + nb, B - b0 - nb, x, o, self.dec_bps, self.sa)
+        main.wait_stream(self.sa)
+        main.wait_stream(self.sb)
+        self.t += 1
+
+
 def run_pace(args, rank: int, world: int):
     import torch
     import bit_recurrent_state_pace_b200 as pace
@@ -317,6 +374,34 @@ def run_pace(args, rank: int, world: int):
         ach, traffic = com_gbs, ncu_traffic("commit", digest)
 
     from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+    lockstep_value = aggregate_rate(BH * P * args.steps, world, elapsed_ms)
+    lockstep_ms = elapsed_ms
+
+    # ---- staggered phases (continuous batching): same work per P steps
+    stag = None
+    if args.schedule == "staggered":
+        dbps, cbps = (int(v) for v in args.stagger_blocks.split(","))
+        stag = Staggered(pace, pool, w, dbps, cbps)
+        stag.preroll(toks, outs, stream)
+        for i in range(args.warmup * P):
+            stag.step(toks[stag.t % P], outs[stag.t % P], stream)
+        torch.cuda.synchronize()
+        assert pool.status() == 0, "device status flags set during the staggered warm-up"
+        barrier(world)
+        torch.cuda.synchronize()
+        sampler = ClockSampler(gpu_uuid)
+        time.sleep(0.2)
+        stag.launches = 0
+        a, b = mk(), mk()
+        a.record(stream)
+        for i in range(args.steps * P):
+            stag.step(toks[stag.t % P], outs[stag.t % P], stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        barrier(world)
+        elapsed_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+        status |= pool.status()
     value = aggregate_rate(BH * P * args.steps, world, elapsed_ms)
 
     # ---- bf16-state comparison path (unquantised, same shape)
@@ -348,7 +433,7 @@ def run_pace(args, rank: int, world: int):
     # ---- end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, pace, pool, w, toks, outs, stream, world, dev)
+        e2e = run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag)
 
     if rank == 0:
         line = {
@@ -371,7 +456,12 @@ def run_pace(args, rank: int, world: int):
             },
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": args.steps * (P + 1),
+            "gpu_launches": stag.launches if stag is not None else args.steps * (P + 1),
+            "schedule": ("staggered: %d slot groups one token apart; each step the full group's "
+                         "commit and decode (stream b) overlap the other groups' decode (stream a), "
+                         "%s blocks per SM" % (P, args.stagger_blocks)) if stag is not None
+                        else "lockstep: every slot at the same phase",
+            "lockstep": {"value": lockstep_value, "ms_per_step": lockstep_ms / args.steps},
             "device_status": status,
             "comparison": compare,
             "cpu_baseline": cpu_base,
@@ -379,9 +469,10 @@ def run_pace(args, rank: int, world: int):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev):
+def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag=None):
     """Same metric through the public API: every step copies its P tokens'
-    inputs host->device from pinned memory and reads every output back."""
+    inputs host->device from pinned memory and reads every output back (in
+    the staggered schedule when one is given)."""
     import torch
     P = w.P
     host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in toks]
@@ -395,9 +486,13 @@ def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev):
             for k, v in host_in[n].items():
                 toks[n][k].copy_(v, non_blocking=True)
             x = toks[n]
-            pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n], sp)
+            if stag is not None:
+                stag.step(x, outs[n], stream)
+            else:
+                pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n], sp)
             host_out[n].copy_(outs[n], non_blocking=True)
-        pace.pace_commit_period(pool.handle, sp)
+        if stag is None:
+            pace.pace_commit_period(pool.handle, sp)
 
     step()
     torch.cuda.synchronize()
