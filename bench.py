@@ -40,6 +40,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["pace", "reference"], default="pace")
     ap.add_argument("--workload", default="concurrency_stress")
     ap.add_argument("--period", type=int, default=None, help="override P")
+    ap.add_argument("--axis", choices=["col", "row"], default=None, help="override the scale axis")
     ap.add_argument("--slots", type=int, default=None, help="override B (smaller profiling case)")
     ap.add_argument("--prefill", type=int, default=None, help="warm-up prefill tokens (default: workload's)")
     ap.add_argument("--e2e-steps", type=int, default=4)
@@ -219,13 +220,21 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, bits):
+L2_BYTES = 126 * 1024 * 1024
+
+
+def workload_config(w, bits, state_bytes=None):
     n8 = sum(1 for b in bits if b == 8)
+    if state_bytes is None or state_bytes >= 4 * L2_BYTES:
+        l2 = "state pool larger than L2 (no flush needed)"
+    else:
+        l2 = (f"state pool {state_bytes / 2**20:.0f} MiB, within 4x of the 126 MB L2: no flush, "
+              "so part of the traffic is served from L2")
     return {"workload": f"{w.name}: B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} P={w.P} "
                         f"{n8}/{w.H} INT8 heads, {w.axis} scales, {w.io_dtype} io",
             "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "P": w.P, "int8_heads": n8,
             "scale_axis": w.axis, "io_dtype": w.io_dtype, "state_dtype": "int4/int8 codes + fp16 scales",
-            "l2": "state pool larger than L2 (no flush needed)", "prefill_tokens": w.warmup}
+            "l2": l2, "prefill_tokens": w.warmup}
 
 
 class Staggered:
@@ -293,6 +302,8 @@ def run_pace(args, rank: int, world: int):
         w = w.replace(warmup=args.prefill)
     if args.slots is not None:
         w = w.replace(B=args.slots)
+    if args.axis is not None:
+        w = w.replace(axis=args.axis)
     bits = pace_synth.head_bits(w, args.seed)
     BH, P = w.B * w.H, w.P
     stream = torch.cuda.current_stream()
@@ -441,7 +452,8 @@ def run_pace(args, rank: int, world: int):
             "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": dict(workload_config(w, bits), parallelism=f"{world} independent pools (no collective)",
+            "config": dict(workload_config(w, bits, int(pool.state.numel())),
+                           parallelism=f"{world} independent pools (no collective)",
                            seq_tokens_per_s=value / w.H),
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                          "frac": ach / hbm, "traffic": traffic, "kernel": dominant,
