@@ -89,11 +89,24 @@ def test_mixed_int8_long_memory_heads():
     print("mixed worst", worst, stats)
 
 
-@pytest.mark.parametrize("P", [1, 2, 4, 16])
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 5, 12, 16])
 def test_period_sweep_small(P):
     w = pace_synth.workload("period_sweep", B=2, H=3, P=P)
     worst, stats = _run_periods(w, periods=2 if P < 16 else 1, random_init=True)
     print("P", P, "worst", worst)
+
+
+@pytest.mark.parametrize("io,axis,d,P", [("f32", "col", 128, 8), ("f32", "row", 64, 16),
+                                         ("bf16", "row", 32, 8), ("bf16", "col", 64, 5),
+                                         ("f32", "col", 32, 3)])
+def test_io_axis_dim_period_matrix(io, axis, d, P):
+    """Mixed 4/8-bit heads across io dtypes, scale axes, head sizes and
+    periods (exact-period and general-period kernels)."""
+    w = pace_synth.workload("mixed_4_8", B=2, H=4, d_k=d, d_v=d, P=P, io_dtype=io, axis=axis,
+                            int8_fraction=0.5)
+    assert 8 in pace_synth.head_bits(w) and 4 in pace_synth.head_bits(w)
+    worst, _ = _run_periods(w, periods=2, random_init=True)
+    print(io, axis, d, P, "worst", worst)
 
 
 @pytest.mark.parametrize("d", [32, 64])
