@@ -17,8 +17,9 @@
 //
 // Design (B200): one CTA per head, one warp per 16-row block; heads strided
 // over a persistent grid, the next head's record, buffered rows, gates and
-// Gram block brought into shared memory by 1-D TMA bulk copies while the
-// current head computes (double buffer, mbarrier completion, bounded waits).
+// Gram block brought into shared memory by 1-D TMA bulk copies two heads
+// ahead (three slots, mbarrier completion, bounded waits), issued by a thread
+// that is otherwise idle during the scale pass.
 // Both contractions run on the f16 tensor cores (mma.sync m16n8k16, fp32
 // accumulation); the codes are exact in f16 and every fp32 operand is split
 // hi + lo after a power-of-two normalisation:
@@ -83,14 +84,15 @@ struct alignas(16) WarpTab {
 template <int D, bool BF16, int PMAX>
 struct alignas(16) Smem {
   using C = Cfg<D, BF16, PMAX>;
-  uint8_t slot[2][C::SLOT];                       // staged record | kv rows | gates | Gram
+  uint8_t slot[3][C::SLOT];                       // staged record | kv rows | gates | Gram
   uint2 bx[C::NTX][C::KS][8][4];                  // X B fragments [tile][ks][g][t]
   uint2 bkf[C::NT][C::KU][8][4];                  // update B fragments [tile][u][g][t]
   float sc[D];                                    // old scales (float)
   float qf[D], sfv[D];                            // new 1/s16 and s16 (column or row)
   float colmax[C::RB][D];
   WarpTab<D> wt[C::RB];
-  uint64_t bar[2];
+  uint64_t bar[3];
+  int hq[3];                                      // head staged in each slot
   float xinv;
   int next_head;
   int slow;
@@ -168,14 +170,12 @@ __device__ __forceinline__ uint32_t magic_exact(float a, float b, float sa, floa
   return (0x6400u | ca) | ((0x6400u | cb) << 16);
 }
 
-__device__ __forceinline__ float pick4(const float4& f, int i) {
-  return i == 0 ? f.x : i == 1 ? f.y : i == 2 ? f.z : f.w;
-}
 
 // EXACT: the pool's period equals PMAX, so every loop bound over tokens is a
 // compile-time constant.
-template <int D, bool BF16, int PMAX, int BITS, bool EXACT>
-__device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot) {
+template <int D, bool BF16, int PMAX, int BITS, bool EXACT, class Issue>
+__device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot,
+                            Issue&& issue_next) {
   using C = Cfg<D, BF16, PMAX>;
   constexpr int KS = C::KS, NT = C::NT, NTX = C::NTX, KU = C::KU, NU = C::NU;
   constexpr int ROWB = D * BITS / 8;
@@ -477,6 +477,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
     }
   }
   __syncthreads();
+  issue_next();   // the issuing thread is idle during the scale pass
   if (col) {
     for (int j = tid; j < D; j += C::THREADS) {
       float a = 0.f;
@@ -577,51 +578,58 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
   // heads [b0 H, (b0 + nb) H) of this launch; n_heads is the end index
   const int first_head = sp.b0 * p.H;
   const int n_heads = (sp.b0 + sp.nb) * p.H;
-  // thread 0 keeps the candidate after the next head and its fill count,
-  // loaded one head ahead so that the load's latency is hidden
+  // thread ISS (idle during the scale pass) issues every bulk copy; it keeps
+  // the candidate head two ahead and its fill count
+  constexpr int ISS = C::THREADS / 2;
   int cand = n_heads, cand_fill = 0;
-  if (tid == 0) {
-    mbar_init(&sm.bar[0], 1);
-    mbar_init(&sm.bar[1], 1);
+  if (tid == ISS) {
+    for (int i = 0; i < 3; ++i) mbar_init(&sm.bar[i], 1);
     fence_mbar_init();
-    sm.slow = 0;
-    const int first = find_full(p, first_head + blockIdx.x, gridDim.x, n_heads);
-    sm.next_head = first;
-    if (first < n_heads) issue_head<D, BF16, PMAX>(p, first, sm, 0);
-    cand = first + gridDim.x;
+    int h = find_full(p, first_head + blockIdx.x, gridDim.x, n_heads);
+    for (int i = 0; i < 3; ++i) sm.hq[i] = n_heads;
+    for (int i = 0; i < 2; ++i) {
+      sm.hq[i] = h;
+      if (h < n_heads) {
+        issue_head<D, BF16, PMAX>(p, h, sm, i);
+        h = find_full(p, h + gridDim.x, gridDim.x, n_heads);
+      }
+    }
+    cand = h;
     if (cand < n_heads) cand_fill = p.fill[cand];
   }
+  if (tid == 0) sm.slow = 0;
   __syncthreads();
-  uint32_t parity[2] = {0u, 0u};
+  uint32_t parity = 0u;
   int s = 0;
-  int head = sm.next_head;
-  while (head < n_heads) {
-    __syncthreads();                      // everyone has read next_head; slot s^1 is free
-    if (tid == 0) {
-      int nxt = cand;
-      if (nxt < n_heads && cand_fill != p.P) nxt = find_full(p, nxt + gridDim.x, gridDim.x, n_heads);
-      sm.next_head = nxt;
-      if (nxt < n_heads) issue_head<D, BF16, PMAX>(p, nxt, sm, s ^ 1);
-      cand = nxt + gridDim.x;
-      if (cand < n_heads) cand_fill = p.fill[cand];
-    }
-    const bool ok = mbar_wait_bounded(&sm.bar[s], parity[s], p.flags);
-    parity[s] ^= 1u;
+  while (true) {
+    const int head = sm.hq[s];
+    if (head >= n_heads) break;
+    const bool ok = mbar_wait_bounded(&sm.bar[s], (parity >> s) & 1u, p.flags);
+    parity ^= 1u << s;
     if (__syncthreads_or(!ok)) {
-      // a copy did not land in time: give the other in-flight copy a bounded
-      // chance to finish before this block's shared memory is released
-      if (tid == 0) mbar_wait_bounded(&sm.bar[s ^ 1], parity[s ^ 1], nullptr);
+      if (tid == ISS)
+        for (int i = 0; i < 3; ++i)
+          if (i != s && sm.hq[i] < n_heads) mbar_wait_bounded(&sm.bar[i], (parity >> i) & 1u, nullptr);
       __syncthreads();
       return;
     }
+    if (tid == 0) sm.slow = 0;   // every thread is past the previous head's encode
+    const int s2 = s == 0 ? 2 : s - 1;   // slot of the head two ahead (held the previous head)
+    auto issue_next = [&]() {
+      if (tid == ISS) {
+        int nxt = cand;
+        if (nxt < n_heads && cand_fill != p.P) nxt = find_full(p, nxt + gridDim.x, gridDim.x, n_heads);
+        sm.hq[s2] = nxt;
+        if (nxt < n_heads) issue_head<D, BF16, PMAX>(p, nxt, sm, s2);
+        cand = nxt < n_heads ? nxt + gridDim.x : n_heads;
+        if (cand < n_heads) cand_fill = p.fill[cand];
+      }
+    };
     if (p.bits[head % p.H] == 4)
-      commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s]);
+      commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s], issue_next);
     else
-      commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s]);
-    __syncthreads();
-    if (tid == 0) sm.slow = 0;
-    head = sm.next_head;
-    s ^= 1;
+      commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s], issue_next);
+    s = s == 2 ? 0 : s + 1;
   }
 }
 
