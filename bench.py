@@ -41,6 +41,9 @@ def parse_args():
     ap.add_argument("--workload", default="concurrency_stress")
     ap.add_argument("--period", type=int, default=None, help="override P")
     ap.add_argument("--axis", choices=["col", "row"], default=None, help="override the scale axis")
+    ap.add_argument("--bits-from-gates", action="store_true",
+                    help="choose the 8-bit heads from the prefill gates (slowest mean decay) "
+                         "instead of the workload's seeded choice")
     ap.add_argument("--slots", type=int, default=None, help="override B (smaller profiling case)")
     ap.add_argument("--prefill", type=int, default=None, help="warm-up prefill tokens (default: workload's)")
     ap.add_argument("--e2e-steps", type=int, default=4)
@@ -314,12 +317,20 @@ def run_pace(args, rank: int, world: int):
         cpu_base = oracle_sample_rate(w, bits, args.cpu_sample_slots, args.seed)
 
     # ---- state: unquantised fp32 prefill, then encode into the pool
-    pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, P, bits, axis=w.axis, io=w.io_dtype, device=dev)
+    io_code = pace.PACE_IO_BF16 if w.io_dtype == "bf16" else pace.PACE_IO_F32
     S = torch.zeros(BH, w.d_v, w.d_k, dtype=torch.float32, device=dev)
+    gates = [] if args.bits_from_gates else None
     for t in range(w.warmup):
         inp = pace_synth.token_inputs(w, t, seed=args.seed + rank, device=dev, phase="warmup")
         pace.pace_gdn_step_f32(S, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
-                               pool.io, None, BH, w.d_k, w.d_v)
+                               io_code, None, BH, w.d_k, w.d_v)
+        if gates is not None:
+            gates.append(inp["alpha"])
+    if gates:
+        rates = pace.pace_decay_rates(torch.stack(gates).contiguous(), w.H, io_code)
+        bits = pace.pace_select_head_bits(rates.cpu().tolist(), sum(1 for b in bits if b == 8))
+        del gates
+    pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, P, bits, axis=w.axis, io=w.io_dtype, device=dev)
     pool.load(S)
     S_bf16 = None if args.no_compare else S.to(torch.bfloat16).view(torch.int16)
     del S
@@ -454,6 +465,9 @@ def run_pace(args, rank: int, world: int):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(workload_config(w, bits, int(pool.state.numel())),
                            parallelism=f"{world} independent pools (no collective)",
+                           int8_head_choice=("slowest mean decay over the prefill gates"
+                                             if args.bits_from_gates else "seeded"),
+                           int8_head_list=[h for h in range(w.H) if bits[h] == 8],
                            seq_tokens_per_s=value / w.H),
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                          "frac": ach / hbm, "traffic": traffic, "kernel": dominant,

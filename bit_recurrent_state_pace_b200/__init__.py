@@ -23,7 +23,8 @@ __all__ = [
     "PACE_FLAG_NONFINITE", "PACE_FLAG_SCALE_OVERFLOW", "PACE_FLAG_BUFFER_FULL", "PACE_FLAG_TIMEOUT",
     "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
     "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
-    "pace_decode_step_range", "pace_commit_period_range",
+    "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
+    "pace_select_head_bits",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -72,6 +73,8 @@ def _load():
         "pace_commit_period": [P, P],
         "pace_decode_step_range": [P, I32, I32, I32, P, P, P, P, P, F32p, P],
         "pace_commit_period_range": [P, I32, I32, I32, P],
+        "pace_decay_rates": [P, I64, I32, I32, P, P],
+        "pace_select_head_bits": [P, I32, I32, P],
         "pace_quantize": [F32p, I64, I32, I32, I32, I32, P, U16p, U32p, P],
         "pace_dequantize": [P, U16p, I64, I32, I32, I32, I32, F32p, P],
         "pace_pool_status": [P, P, ctypes.POINTER(ctypes.c_uint32)],
@@ -174,6 +177,27 @@ def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
 
 def pace_commit_period(handle: int, stream=None) -> None:
     _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_decay_rates(alpha: torch.Tensor, num_heads: int, io: int, rates: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Mean -ln(alpha) per head over the rows of a device gate matrix [rows][num_heads]."""
+    if rates is None:
+        rates = torch.empty(num_heads, dtype=torch.float64, device=alpha.device)
+    rows = alpha.numel() // num_heads
+    _check("pace_decay_rates", lib.pace_decay_rates(_ptr(alpha), rows, num_heads, io, _ptr(rates),
+                                                     _stream(stream)))
+    return rates
+
+
+def pace_select_head_bits(rates: Sequence[float], num_int8: int) -> list:
+    """Host: 8 bits for the num_int8 heads with the slowest decay, 4 for the rest."""
+    vals = [float(r) for r in rates]
+    arr = (ctypes.c_double * max(len(vals), 1))(*vals)
+    out = (ctypes.c_uint8 * max(len(vals), 1))()
+    _check("pace_select_head_bits", lib.pace_select_head_bits(
+        ctypes.cast(arr, ctypes.c_void_p), len(vals), num_int8, ctypes.cast(out, ctypes.c_void_p)))
+    return [int(out[i]) for i in range(len(vals))]
 
 
 def pace_decode_step_range(handle: int, slot_begin: int, slot_count: int, blocks_per_sm: int,

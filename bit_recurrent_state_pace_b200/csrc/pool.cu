@@ -298,4 +298,42 @@ pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const 
                                               as_stream(stream)));
 }
 
+pace_status pace_decay_rates(const void* alpha, int64_t rows, int32_t num_heads, int32_t io_dtype,
+                             double* rates, void* stream) {
+  if (!alpha || !rates || rows < 0 || num_heads < 1 || num_heads > PACE_MAX_HEADS)
+    return PACE_ERR_INVALID_ARG;
+  if (io_dtype != PACE_IO_BF16 && io_dtype != PACE_IO_F32) return PACE_ERR_INVALID_ARG;
+  if (!aligned(alpha, io_dtype == PACE_IO_BF16 ? 2 : 4) || !aligned(rates, 8)) return PACE_ERR_INVALID_ARG;
+  return from_cuda(pace::launch_decay_rates(alpha, rows, num_heads, io_dtype, rates, as_stream(stream)));
+}
+
+pace_status pace_select_head_bits(const double* rates, int32_t num_heads, int32_t num_int8,
+                                  uint8_t* head_bits) {
+  if (!rates || !head_bits || num_heads < 1 || num_heads > PACE_MAX_HEADS || num_int8 < 0 ||
+      num_int8 > num_heads)
+    return PACE_ERR_INVALID_ARG;
+  int order[PACE_MAX_HEADS];
+  for (int h = 0; h < num_heads; ++h) order[h] = h;
+  // slowest decay first; NaN rates last; ties by head index (stable)
+  auto before = [&](int a, int b) {
+    const double ra = rates[a], rb = rates[b];
+    const bool na = ra != ra, nb = rb != rb;
+    if (na != nb) return nb;
+    if (!na && ra != rb) return ra < rb;
+    return a < b;
+  };
+  for (int i = 1; i < num_heads; ++i) {   // insertion sort: H <= 256
+    const int x = order[i];
+    int j = i - 1;
+    while (j >= 0 && before(x, order[j])) {
+      order[j + 1] = order[j];
+      --j;
+    }
+    order[j + 1] = x;
+  }
+  for (int h = 0; h < num_heads; ++h) head_bits[h] = 4;
+  for (int i = 0; i < num_int8; ++i) head_bits[order[i]] = 8;
+  return PACE_OK;
+}
+
 }  // extern "C"

@@ -228,6 +228,31 @@ pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const 
                                const void* alpha, const void* beta, int32_t io_dtype,
                                float* o, int64_t n, int32_t d_k, int32_t d_v, void* stream);
 
+/*
+ * Choosing the 8-bit heads from their gates ([P2] paragraph on 8-bit
+ * precision for selected heads; [P4] TL;DR (3): heads whose errors persist,
+ * the long-memory heads, are kept at 8 bits).
+ *
+ * pace_decay_rates: alpha is a device matrix [rows][num_heads] in io_dtype
+ * (e.g. the gates of a calibration prefill, rows = tokens x sequences);
+ * rates (device, num_heads doubles, overwritten) receives each head's mean
+ * decay rate  r_h = (1/rows) sum_rows -ln(alpha[row][h]), accumulated in
+ * fp64.  A smaller rate is a longer memory.  Gates <= 0 or NaN give +inf or
+ * NaN rates.  Asynchronous on `stream`.
+ *
+ * pace_select_head_bits (host only): head_bits[h] = 8 for the num_int8 heads
+ * with the smallest rates (NaN rates last, ties to the lower head index),
+ * 4 for the others -- ready for pace_pool_desc.head_bits.
+ *
+ * Neither call has a counterpart in the pages' text beyond the statement
+ * that long-memory heads get 8 bits; the statistic is this library's
+ * reading.
+ */
+pace_status pace_decay_rates(const void* alpha, int64_t rows, int32_t num_heads, int32_t io_dtype,
+                             double* rates, void* stream);
+pace_status pace_select_head_bits(const double* rates, int32_t num_heads, int32_t num_int8,
+                                  uint8_t* head_bits);
+
 /* Human-readable name of a status code (static string). */
 const char* pace_status_string(pace_status s);
 

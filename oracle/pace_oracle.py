@@ -42,6 +42,8 @@ Pages cited (by title and section):
 5. Mixed heads.  [P2] "Additionally, PACE uses 8-bit precision ..." paragraph,
    [P4] TL;DR (3) and the flowchart's "long-memory heads -> 8-bit heads":
    per-head bit widths, handled by calling ``quantize`` with bits 4 or 8.
+   ``decay_rates`` / ``select_head_bits`` choose the 8-bit heads from the
+   gates (mean -ln alpha per head, the slowest-decaying heads first).
 
 Everything here is fp64 except the quantiser, which takes the fp32 state and
 reproduces the fp32/fp16 operations of the encoding one by one with numpy's
@@ -380,3 +382,29 @@ def relative_error(o_test, o_ref) -> np.ndarray:
     num = np.max(np.abs(o_test - o_ref), axis=-1)
     den = np.maximum(np.max(np.abs(o_ref), axis=-1), 1e-6)
     return num / den
+
+
+# --------------------------------------------------------------------------
+# Which heads keep 8 bits.  [P2] (paragraph on 8-bit precision for selected
+# heads) and [P4] TL;DR (3): heads whose errors persist -- long-memory heads
+# -- are stored at 8 bits.  Reading: a head's memory is set by its gate, a
+# write decaying by alpha per token, so heads are ranked by their mean decay
+# rate -ln(alpha) over a calibration stream (smaller = longer memory).
+# --------------------------------------------------------------------------
+
+def decay_rates(alpha) -> np.ndarray:
+    """Mean of -ln(alpha) over the leading axes, per head (last axis), fp64."""
+    a = np.asarray(alpha, dtype=np.float64)
+    a = a.reshape(-1, a.shape[-1])
+    return np.mean(-np.log(a), axis=0)
+
+
+def select_head_bits(rates, num_int8: int) -> List[int]:
+    """8 bits for the num_int8 heads with the smallest rate (NaN last, ties to
+    the lower head index), 4 bits for the rest."""
+    r = [float(x) for x in rates]
+    order = sorted(range(len(r)), key=lambda h: (np.isnan(r[h]), 0.0 if np.isnan(r[h]) else r[h], h))
+    bits = [4] * len(r)
+    for h in order[:num_int8]:
+        bits[h] = 8
+    return bits
