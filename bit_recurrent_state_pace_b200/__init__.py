@@ -24,7 +24,7 @@ __all__ = [
     "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
     "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
     "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
-    "pace_select_head_bits",
+    "pace_select_head_bits", "pace_prefill", "pace_prefill_range",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -74,6 +74,8 @@ def _load():
         "pace_decode_step_range": [P, I32, I32, I32, P, P, P, P, P, F32p, P],
         "pace_commit_period_range": [P, I32, I32, I32, P],
         "pace_decay_rates": [P, I64, I32, I32, P, P],
+        "pace_prefill": [P, I64, P, P, P, P, P, F32p, P],
+        "pace_prefill_range": [P, I32, I32, I64, P, P, P, P, P, F32p, P],
         "pace_select_head_bits": [P, I32, I32, P],
         "pace_quantize": [F32p, I64, I32, I32, I32, I32, P, U16p, U32p, P],
         "pace_dequantize": [P, U16p, I64, I32, I32, I32, I32, F32p, P],
@@ -177,6 +179,18 @@ def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
 
 def pace_commit_period(handle: int, stream=None) -> None:
     _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_prefill(handle: int, T: int, q, k, v, alpha, beta, o=None, stream=None) -> None:
+    _check("pace_prefill", lib.pace_prefill(handle, T, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                             _ptr(beta), _ptr(o), _stream(stream)))
+
+
+def pace_prefill_range(handle: int, slot_begin: int, slot_count: int, T: int, q, k, v, alpha, beta,
+                       o=None, stream=None) -> None:
+    _check("pace_prefill_range", lib.pace_prefill_range(handle, slot_begin, slot_count, T, _ptr(q),
+                                                         _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                                         _ptr(o), _stream(stream)))
 
 
 def pace_decay_rates(alpha: torch.Tensor, num_heads: int, io: int, rates: Optional[torch.Tensor] = None,
@@ -321,6 +335,11 @@ class PacePool:
                           stream=None) -> torch.Tensor:
         pace_decode_step_range(self.handle, slot_begin, slot_count, blocks_per_sm, q, k, v, alpha,
                                beta, o, stream)
+        return o
+
+    def prefill(self, q, k, v, alpha, beta, o=None, stream=None) -> Optional[torch.Tensor]:
+        """T tokens [T][B][H][d] through the chunked fp32 prefill; returns o."""
+        pace_prefill(self.handle, int(q.shape[0]), q, k, v, alpha, beta, o, stream)
         return o
 
     def commit_period_range(self, slot_begin, slot_count, blocks_per_sm=0, stream=None) -> None:

@@ -33,9 +33,8 @@
 // f16 magic-number conversion (1032 + c, 1152 + c) and packed in place.
 #include <type_traits>
 
-#include "encode.cuh"
-#include "frag.cuh"
 #include "tma.cuh"
+#include "update_common.cuh"
 
 namespace pace {
 
@@ -43,16 +42,6 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 
-// floor(log2(m)) for a positive normal float, from its exponent bits
-__device__ __forceinline__ int exp2_floor(float m) { return (int)((__float_as_uint(m) >> 23) & 0xffu) - 127; }
-// 2^e for e in [-126, 127], exact
-__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
-
-__device__ __forceinline__ float max_nan(float a, float b) {
-  float r;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-  return r;
-}
 
 template <int D, bool BF16, int PMAX>
 struct Cfg {
@@ -125,10 +114,6 @@ __device__ __forceinline__ void issue_head(const PoolDev& p, int head, Smem<D, B
   tma_load_1d(dst + C::REC + C::KVB + C::ABB, gr, p.gram_stride, &sm.bar[s]);
 }
 
-__device__ __forceinline__ float io_at(const uint8_t* base, int idx, bool bf16) {
-  if (bf16) return __uint_as_float(((uint32_t)reinterpret_cast<const uint16_t*>(base)[idx]) << 16);
-  return reinterpret_cast<const float*>(base)[idx];
-}
 
 // Codes of rows 16r+g, 16r+g+8 for lane (g, t), read from shared memory.
 template <int D, int BITS>
@@ -155,20 +140,6 @@ __device__ __forceinline__ void load_rows_smem(RowBlock<D, BITS>& rb, const uint
   }
 }
 
-template <int BITS>
-__device__ __forceinline__ uint32_t magic_fast(float a, float b, float qa, float qb) {
-  const float M = BITS == 4 ? 1032.f : 1152.f;
-  const float2 r = __ffma2_rn(make_float2(a, b), make_float2(qa, qb), make_float2(M, M));
-  return h2u(__floats2half2_rn(r.x, r.y));
-}
-
-template <int BITS>
-__device__ __forceinline__ uint32_t magic_exact(float a, float b, float sa, float sb) {
-  const int qmax = BITS == 4 ? 7 : 127, off = BITS == 4 ? 8 : 128;
-  const uint32_t ca = (uint32_t)(encode_value(a, sa, qmax) + off);
-  const uint32_t cb = (uint32_t)(encode_value(b, sb, qmax) + off);
-  return (0x6400u | ca) | ((0x6400u | cb) << 16);
-}
 
 
 // EXACT: the pool's period equals PMAX, so every loop bound over tokens is a

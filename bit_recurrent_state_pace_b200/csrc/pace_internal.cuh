@@ -102,6 +102,9 @@ cudaError_t launch_decode_step(const PoolDev& p, const Span& sp, const void* q, 
                                const void* v, const void* alpha, const void* beta, float* o,
                                cudaStream_t st);
 cudaError_t launch_commit(const PoolDev& p, const Span& sp, cudaStream_t st);
+cudaError_t launch_prefill(const PoolDev& p, const Span& sp, int64_t T, const void* q,
+                           const void* k, const void* v, const void* alpha, const void* beta,
+                           float* o, cudaStream_t st);
 cudaError_t launch_decay_rates(const void* alpha, int64_t rows, int H, int io, double* rates,
                                cudaStream_t st);
 cudaError_t launch_gdn_step_f32(float* S, const void* q, const void* k, const void* v,

@@ -222,6 +222,25 @@ pace_status pace_commit_period_range(pace_pool* pool, int32_t slot_begin, int32_
   return from_cuda(pace::launch_commit(pool->dev, sp, as_stream(stream)));
 }
 
+pace_status pace_prefill_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
+                               int64_t T, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* beta, float* o, void* stream) {
+  if (!pool || T < 0 || (T > 0 && (!q || !k || !v || !alpha || !beta))) return PACE_ERR_INVALID_ARG;
+  if (!span_ok(pool, slot_begin, slot_count, 0)) return PACE_ERR_INVALID_ARG;
+  const size_t esz = pool->dev.io == PACE_IO_BF16 ? 2 : 4;
+  if (!aligned(q, esz) || !aligned(k, esz) || !aligned(v, esz) || !aligned(alpha, esz) ||
+      !aligned(beta, esz) || !aligned(o, 4))
+    return PACE_ERR_INVALID_ARG;
+  const pace::Span sp{slot_begin, slot_count, 0};
+  return from_cuda(pace::launch_prefill(pool->dev, sp, T, q, k, v, alpha, beta, o, as_stream(stream)));
+}
+
+pace_status pace_prefill(pace_pool* pool, int64_t T, const void* q, const void* k, const void* v,
+                         const void* alpha, const void* beta, float* o, void* stream) {
+  if (!pool) return PACE_ERR_INVALID_ARG;
+  return pace_prefill_range(pool, 0, pool->dev.B, T, q, k, v, alpha, beta, o, stream);
+}
+
 pace_status pace_commit_period(pace_pool* pool, void* stream) {
   if (!pool) return PACE_ERR_INVALID_ARG;
   return pace_commit_period_range(pool, 0, pool->dev.B, 0, stream);

@@ -229,6 +229,26 @@ pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const 
                                float* o, int64_t n, int32_t d_k, int32_t d_v, void* stream);
 
 /*
+ * Chunked fp32 prefill (the chunked prefill kernels that [P2] "Periodic
+ * Rounding" cites; [P4] flowchart "State update, chunked, high precision").
+ * For every head of the slots (all of them, or [slot_begin, slot_begin +
+ * slot_count)) whose buffer is empty: start from the stored state, apply T
+ * tokens exactly in fp32 in chunks of 8 (UT/WY form), write every token's
+ * output, and encode the final state into the pool once, at the end (fresh
+ * absmax scales at the head's bit width); the buffer stays empty.
+ *   q, k: [T][num_slots][num_heads][d_k], v: [T][num_slots][num_heads][d_v],
+ *   alpha, beta: [T][num_slots][num_heads], all io_dtype, device, aligned
+ *   to the element size; o: fp32 [T][num_slots][num_heads][d_v] or NULL.
+ * A head with buffered tokens is skipped (PACE_FLAG_BUFFER_FULL).  A pool
+ * that starts from zeros (all codes and scales 0) prefills from S = 0.
+ */
+pace_status pace_prefill(pace_pool* pool, int64_t T, const void* q, const void* k, const void* v,
+                         const void* alpha, const void* beta, float* o, void* stream);
+pace_status pace_prefill_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
+                               int64_t T, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* beta, float* o, void* stream);
+
+/*
  * Choosing the 8-bit heads from their gates ([P2] paragraph on 8-bit
  * precision for selected heads; [P4] TL;DR (3): heads whose errors persist,
  * the long-memory heads, are kept at 8 bits).
