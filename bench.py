@@ -41,6 +41,8 @@ def parse_args():
     ap.add_argument("--workload", default="concurrency_stress")
     ap.add_argument("--period", type=int, default=None, help="override P")
     ap.add_argument("--axis", choices=["col", "row"], default=None, help="override the scale axis")
+    ap.add_argument("--prefill-tokens", type=int, default=64,
+                    help="tokens of the chunked fp32 prefill measured after the decode (0: skip)")
     ap.add_argument("--bits-from-gates", action="store_true",
                     help="choose the 8-bit heads from the prefill gates (slowest mean decay) "
                          "instead of the workload's seeded choice")
@@ -457,6 +459,33 @@ def run_pace(args, rank: int, world: int):
     if not args.no_e2e:
         e2e = run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag)
 
+    # ---- chunked fp32 prefill of T tokens into the whole pool (after the decode
+    #      numbers: it rewrites the pool); not part of the headline step
+    prefill = None
+    if args.prefill_tokens > 0 and stag is None:
+        Tp = args.prefill_tokens
+        ptoks = [pace_synth.token_inputs(w, 100000 + t, seed=args.seed + rank, device=dev) for t in range(Tp)]
+        pin = {key: torch.stack([x[key] for x in ptoks]).contiguous() for key in ptoks[0]}
+        del ptoks
+        po = torch.empty(Tp, w.B, w.H, w.d_v, dtype=torch.float32, device=dev)
+        pool.prefill(pin["q"], pin["k"], pin["v"], pin["alpha"], pin["beta"], po)   # warm-up call
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = mk(), mk()
+        a.record(stream)
+        pool.prefill(pin["q"], pin["k"], pin["v"], pin["alpha"], pin["beta"], po)
+        b.record(stream)
+        torch.cuda.synchronize()
+        pms = max_over_ranks(a.elapsed_time(b), world, dev)
+        esz = 2 if w.io_dtype == "bf16" else 4
+        pbytes = (Tp * BH * ((2 * w.d_k + w.d_v + 2) * esz + 4 * w.d_v) + 2 * int(pool.state.numel()))
+        from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+        prefill = {"tokens": Tp, "value": aggregate_rate(BH * Tp, world, pms), "unit": "head-tokens/s",
+                   "ms": pms, "alg_bytes": pbytes, "achieved_gbs": pbytes / (pms * 1e-3) / 1e9,
+                   "frac_of_peak": pbytes / (pms * 1e-3) / 1e9 / measured_peaks()[0],
+                   "status": pool.status()}
+        del pin, po
+
     if rank == 0:
         line = {
             "metric": "decode head-tokens/s (B x H heads, 4-bit state, P=%d)" % P,
@@ -490,6 +519,7 @@ def run_pace(args, rank: int, world: int):
             "lockstep": {"value": lockstep_value, "ms_per_step": lockstep_ms / args.steps},
             "device_status": status,
             "comparison": compare,
+            "prefill": prefill,
             "cpu_baseline": cpu_base,
         }
         print(json.dumps(line), flush=True)
