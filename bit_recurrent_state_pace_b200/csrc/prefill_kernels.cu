@@ -44,20 +44,47 @@ struct PCfg {
 template <int D, bool BF16>
 struct alignas(16) PSmem {
   using C = PCfg<D, BF16>;
-  float kq[2][CH][D];                 // chunk keys [0] and queries [1], fp32
-  float vv[CH][D];                    // chunk values
+  // chunk rows k [0], q [1], v [2] in the io dtype, double-buffered: chunk
+  // c + 1 arrives by asynchronous copies while chunk c computes
+  uint8_t raw[2][3][CH][D * (BF16 ? 2 : 4)];
+  float abuf[2][2][CH];               // [buffer][alpha, beta][token]
   uint2 bx[C::NKX][C::KS][8][4];      // K / Q B fragments [tile][ks][g][t]
   uint2 bkf[C::NT][C::KU][8][4];      // update B fragments [tile][u][g][t]
   float G[CH][CH], M[CH][CH];         // k_t.k_s and q_t.k_s
   float TB[CH][CH];                   // T[s][s'] beta_s'
   float MW[CH][CH];                   // gamma_{t/s} q_t.k_s for s <= t
-  float gam[CH], suf[CH], al[CH], be[CH];
+  float gam[CH], suf[CH];
   float sc[D];                        // stored scales, then new 1/s16 and s16
   float qf[D], sfv[D];
   float colmax[C::RB][D];
   float4 wq[C::RB][C::KS][4];         // per-warp quantisation factors in fragment order
   int slow;
 };
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Issue the asynchronous copies of chunk rows [c0, c0 + n) of k, q, v for
+// `head` into staging buffer `buf` (16-byte pieces over the block's threads).
+template <int D, bool BF16, class SM>
+__device__ __forceinline__ void stage_chunk(SM& sm, int buf, int64_t c0, int n, int64_t BH, int head,
+                                            const void* q, const void* k, const void* v, int nthreads) {
+  constexpr int RBYTES = D * (BF16 ? 2 : 4);
+  constexpr int PIECES = RBYTES / 16;
+  for (int it = threadIdx.x; it < 3 * n * PIECES; it += nthreads) {
+    const int which = it / (n * PIECES), rem = it - which * n * PIECES;
+    const int s = rem / PIECES, pc = rem - s * PIECES;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(which == 0 ? k : which == 1 ? q : v) +
+                         (size_t)((c0 + s) * BH + head) * RBYTES + 16 * pc;
+    cp_async16(&sm.raw[buf][which][s][16 * pc], src);
+  }
+  cp_async_commit();
+}
 
 // Lane L ends with the warp-wide sum of value index (L mod V).
 template <int V>
@@ -125,28 +152,40 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
   float F = 1.f;   // acc = F * S
 
   // ---- chunks ----------------------------------------------------------------
-  for (int64_t c0 = 0; c0 < T; c0 += CH) {
+  const int io = BF16 ? PACE_IO_BF16 : PACE_IO_F32;
+  auto kq = [&](int buf, int which, int s, int e) -> float { return io_at(sm.raw[buf][which][s], e, BF16); };
+  // chunk 0: rows by asynchronous copy, gates directly
+  if (T > 0) stage_chunk<D, BF16>(sm, 0, 0, T < CH ? (int)T : CH, BH, head, q, k, v, C::THREADS);
+  if (tid < CH) {
+    const bool in = tid < T;
+    const size_t row = (size_t)(tid * BH + head);
+    sm.abuf[0][0][tid] = in ? load_io(alpha, row, io) : 1.f;
+    sm.abuf[0][1][tid] = in ? load_io(beta, row, io) : 0.f;
+  }
+  int buf = 0;
+  for (int64_t c0 = 0; c0 < T; c0 += CH, buf ^= 1) {
     const int n = (int)((T - c0) < CH ? (T - c0) : CH);
-    __syncthreads();   // previous chunk's tables and scalars are no longer read
-    // a. stage the chunk's k, q, v (fp32) and gates; tokens >= n read as zero
-    for (int idx = tid; idx < 3 * CH * D; idx += C::THREADS) {
-      const int which = idx / (CH * D), rem = idx - which * CH * D, s = rem / D, e = rem - s * D;
-      float val = 0.f;
-      if (s < n) {
-        const size_t row = (size_t)((c0 + s) * BH + head) * D + e;
-        const void* src = which == 0 ? k : which == 1 ? q : v;
-        val = load_io(src, row, BF16 ? PACE_IO_BF16 : PACE_IO_F32);
-      }
-      if (which < 2) sm.kq[which][s][e] = val;
-      else sm.vv[s][e] = val;
+    cp_async_wait_all();
+    // rows past the last token read as zero
+    for (int idx = tid; idx < 3 * (CH - n) * D; idx += C::THREADS) {
+      const int which = idx / ((CH - n) * D), rem = idx - which * (CH - n) * D;
+      const int s = n + rem / D, e = rem % D;
+      if (BF16) reinterpret_cast<uint16_t*>(sm.raw[buf][which][s])[e] = 0;
+      else reinterpret_cast<float*>(sm.raw[buf][which][s])[e] = 0.f;
     }
-    if (tid < CH) {
-      const bool in = tid < n;
-      const size_t row = (size_t)((c0 + tid) * BH + head);
-      sm.al[tid] = in ? load_io(alpha, row, BF16 ? PACE_IO_BF16 : PACE_IO_F32) : 1.f;
-      sm.be[tid] = in ? load_io(beta, row, BF16 ? PACE_IO_BF16 : PACE_IO_F32) : 0.f;
+    __syncthreads();   // chunk c staged; the previous chunk's readers are done
+    // chunk c + 1: rows now (asynchronous), gates into registers of the last
+    // warp's first lanes, stored before the chunk ends
+    const int64_t c1 = c0 + CH;
+    const int n1 = c1 < T ? (int)((T - c1) < CH ? (T - c1) : CH) : 0;
+    if (n1 > 0) stage_chunk<D, BF16>(sm, buf ^ 1, c1, n1, BH, head, q, k, v, C::THREADS);
+    const int gl = tid - (C::THREADS - 32);   // lane of the last warp
+    float a_nx = 1.f, b_nx = 0.f;
+    if (gl >= 0 && gl < CH && gl < n1) {
+      const size_t row = (size_t)((c1 + gl) * BH + head);
+      a_nx = load_io(alpha, row, io);
+      b_nx = load_io(beta, row, io);
     }
-    __syncthreads();
 
     // b. dot products in groups of 16 (G: 0..63, M: 64..127), groups strided over warps
     for (int base = 16 * w; base < 2 * CH * CH; base += 16 * C::RB) {
@@ -155,11 +194,9 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       for (int d = 0; d < 16; ++d) {
         const int dd = base + d;
         const int which = dd / (CH * CH), tt = (dd / CH) % CH, ss = dd % CH;
-        const float* va = sm.kq[which][tt];
-        const float* vb = sm.kq[0][ss];
         float a = 0.f;
 #pragma unroll
-        for (int e = lane; e < D; e += 32) a = fmaf(va[e], vb[e], a);
+        for (int e = lane; e < D; e += 32) a = fmaf(kq(buf, which, tt, e), kq(buf, 0, ss, e), a);
         part[d] = a;
       }
       const float r = transpose_sum<16>(part, lane);
@@ -170,22 +207,25 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
         else sm.M[tt][ss] = r;
       }
     }
+    __syncthreads();   // dot products ready
+    // warps 1.. build the operand tables while warp 0 forms the chunk scalars
+    const int tbl_tid = tid - 32, tbl_n = C::THREADS - 32;
     // K / Q B-fragment tables: entry (x, ks, g, t) of tile x (K, Q, K_lo, Q_lo)
     // holds channels jof(t, ks, 0..3) of token g
-    for (int it = tid; it < NKX * KS * 32; it += C::THREADS) {
+    for (int it = tbl_tid; tbl_tid >= 0 && it < NKX * KS * 32; it += tbl_n) {
       const int tt = it & 3, gg = (it >> 2) & 7, xk = it >> 5;
       const int ks = xk % KS, x = xk / KS;
       __half hv[4];
 #pragma unroll
       for (int pos = 0; pos < 4; ++pos) {
-        const float val = sm.kq[x & 1][gg][jof<D, BITS>(tt, ks, pos)];
+        const float val = kq(buf, x & 1, gg, jof<D, BITS>(tt, ks, pos));
         const __half hi = __float2half_rn(val);
         hv[pos] = x < 2 ? hi : __float2half_rn(val - __half2float(hi));
       }
       sm.bx[x][ks][gg][tt] = make_uint2(h2u(__halves2half2(hv[0], hv[1])), h2u(__halves2half2(hv[2], hv[3])));
     }
     // update B table, as in the period commit (slots: token sigma % CH of segment sigma / CH)
-    for (int it = tid; it < NT * KU * 32; it += C::THREADS) {
+    for (int it = tbl_tid; tbl_tid >= 0 && it < NT * KU * 32; it += tbl_n) {
       const int tt = it & 3, gg = (it >> 2) & 7, tu = it >> 5;
       const int u = tu % KU, tau = tu / KU;
       const int j = jof<D, BITS>(gg >> 1, tau >> 1, 2 * (tau & 1) + (gg & 1));
@@ -199,7 +239,7 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
           const int seg = sigma / CH, s2 = sigma % CH;
           __half hh = __ushort_as_half((unsigned short)0);
           if (seg < C::NSEG) {
-            const float kv = sm.kq[0][s2][j];
+            const float kv = kq(buf, 0, s2, j);
             hh = __float2half_rn(kv);
             if (seg == 2) hh = __float2half_rn(kv - __half2float(hh));
           }
@@ -209,12 +249,11 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       }
       sm.bkf[tau][u][gg][tt] = make_uint2(wv[0], wv[1]);
     }
-    __syncthreads();
 
     // c. chunk scalars, lane s = token s (warp 0)
     if (w == 0) {
       const bool in = lane < n;
-      const float al = in ? sm.al[lane] : 1.f, be = in ? sm.be[lane] : 0.f;
+      const float al = in ? sm.abuf[buf][0][lane] : 1.f, be = in ? sm.abuf[buf][1][lane] : 0.f;
       float gcum = al;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -313,8 +352,8 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       for (int e = 0; e < 2; ++e) {
         const int s = 2 * t + e;
         const float gs = sm.gam[s];
-        ro[e][0] = sm.vv[s][i0] - gs * (xk[e] * inv);
-        ro[e][1] = sm.vv[s][i1] - gs * (xk[2 + e] * inv);
+        ro[e][0] = kq(buf, 2, s, i0) - gs * (xk[e] * inv);
+        ro[e][1] = kq(buf, 2, s, i1) - gs * (xk[2 + e] * inv);
       }
 #pragma unroll
       for (int src = 0; src < 4; ++src)
@@ -413,6 +452,10 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
         const uint2 bb = sm.bkf[tau][uu][g][t];
         mma16816(acc[tau], Au[uu], bb.x, bb.y);
       }
+    if (gl >= 0 && gl < CH) {
+      sm.abuf[buf ^ 1][0][gl] = a_nx;
+      sm.abuf[buf ^ 1][1][gl] = b_nx;
+    }
   }
 
   // ---- encode the final state (acc = F S) --------------------------------------
