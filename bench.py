@@ -527,28 +527,31 @@ def run_pace(args, rank: int, world: int):
 
 def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag=None):
     """Same metric through the public API: every step copies its P tokens'
-    inputs host->device from pinned memory and reads every output back (in
-    the staggered schedule when one is given)."""
+    inputs host->device from pinned memory and reads every output back.  In
+    lockstep this is one pace_decode_host call per period (copies of token
+    t+1 in and t-1 out overlap token t's kernels); the staggered schedule
+    copies and computes token by token on one stream."""
     import torch
     P = w.P
-    host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in toks]
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h2d = sum(v.numel() * v.element_size() for t in host_in for v in t.values())
-    d2h = sum(o.numel() * o.element_size() for o in host_out)
-    sp = stream.cuda_stream
+    host_out = torch.empty((P,) + tuple(outs[0].shape), dtype=outs[0].dtype).pin_memory()
+    if stag is None:
+        host_in = {k: torch.stack([t[k].cpu() for t in toks]).contiguous().pin_memory() for k in toks[0]}
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    else:
+        host_in = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in toks]
+        h2d = sum(v.numel() * v.element_size() for t in host_in for v in t.values())
+    d2h = host_out.numel() * host_out.element_size()
 
     def step():
+        if stag is None:
+            pool.decode_host(host_in["q"], host_in["k"], host_in["v"], host_in["alpha"],
+                             host_in["beta"], host_out, stream)
+            return
         for n in range(P):
             for k, v in host_in[n].items():
                 toks[n][k].copy_(v, non_blocking=True)
-            x = toks[n]
-            if stag is not None:
-                stag.step(x, outs[n], stream)
-            else:
-                pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n], sp)
+            stag.step(toks[n], outs[n], stream)
             host_out[n].copy_(outs[n], non_blocking=True)
-        if stag is None:
-            pace.pace_commit_period(pool.handle, sp)
 
     step()
     torch.cuda.synchronize()

@@ -24,7 +24,8 @@ __all__ = [
     "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
     "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
     "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
-    "pace_select_head_bits", "pace_prefill", "pace_prefill_range",
+    "pace_select_head_bits", "pace_prefill", "pace_prefill_range", "pace_host_staging_bytes",
+    "pace_decode_host",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -75,6 +76,8 @@ def _load():
         "pace_commit_period_range": [P, I32, I32, I32, P],
         "pace_decay_rates": [P, I64, I32, I32, P, P],
         "pace_prefill": [P, I64, P, P, P, P, P, F32p, P],
+        "pace_host_staging_bytes": [P, Sp],
+        "pace_decode_host": [P, I32, P, P, P, P, P, P, P, P, P, P],
         "pace_prefill_range": [P, I32, I32, I64, P, P, P, P, P, F32p, P],
         "pace_select_head_bits": [P, I32, I32, P],
         "pace_quantize": [F32p, I64, I32, I32, I32, I32, P, U16p, U32p, P],
@@ -179,6 +182,27 @@ def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
 
 def pace_commit_period(handle: int, stream=None) -> None:
     _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_host_staging_bytes(handle: int) -> int:
+    n = ctypes.c_size_t()
+    _check("pace_host_staging_bytes", lib.pace_host_staging_bytes(handle, ctypes.byref(n)))
+    return n.value
+
+
+def _host_ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("pace_decode_host takes contiguous host tensors")
+    return t.data_ptr()
+
+
+def pace_decode_host(handle: int, n_tokens: int, q, k, v, alpha, beta, o, staging, stream,
+                     h2d_stream, d2h_stream) -> None:
+    _check("pace_decode_host", lib.pace_decode_host(
+        handle, n_tokens, _host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(alpha), _host_ptr(beta),
+        _host_ptr(o), _ptr(staging), _stream(stream), _stream(h2d_stream), _stream(d2h_stream)))
 
 
 def pace_prefill(handle: int, T: int, q, k, v, alpha, beta, o=None, stream=None) -> None:
@@ -341,6 +365,19 @@ class PacePool:
         """T tokens [T][B][H][d] through the chunked fp32 prefill; returns o."""
         pace_prefill(self.handle, int(q.shape[0]), q, k, v, alpha, beta, o, stream)
         return o
+
+    def decode_host(self, q, k, v, alpha, beta, o=None, stream=None) -> None:
+        """T decode steps (each followed by the commit of full heads) from host
+        tensors [T][B][H][d]; outputs land in the host tensor o (fp32
+        [T][B][H][d_v], pinned for full speed) once `stream` completes."""
+        if getattr(self, "_staging", None) is None:
+            self._staging = torch.empty(pace_host_staging_bytes(self.handle), dtype=torch.uint8,
+                                        device=self.state.device)
+            self._h2d = torch.cuda.Stream(self.state.device)
+            self._d2h = torch.cuda.Stream(self.state.device)
+        s = stream if stream is not None else torch.cuda.current_stream(self.state.device)
+        pace_decode_host(self.handle, int(q.shape[0]), q, k, v, alpha, beta, o, self._staging, s,
+                         self._h2d, self._d2h)
 
     def commit_period_range(self, slot_begin, slot_count, blocks_per_sm=0, stream=None) -> None:
         pace_commit_period_range(self.handle, slot_begin, slot_count, blocks_per_sm, stream)

@@ -9,6 +9,10 @@ struct pace_pool {
   pace_pool_desc desc;
   size_t state_bytes, buffer_bytes, aux_bytes, kv_bytes;
   size_t rec_bytes[PACE_MAX_HEADS];
+  // pace_decode_host: per staging slot, the event of its last output copy,
+  // and the staging buffer they refer to
+  cudaEvent_t host_done[2] = {nullptr, nullptr};
+  const void* host_staging = nullptr;
 };
 
 namespace {
@@ -168,7 +172,12 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
   return PACE_OK;
 }
 
-void pace_destroy_pool(pace_pool* pool) { delete pool; }
+void pace_destroy_pool(pace_pool* pool) {
+  if (!pool) return;
+  for (cudaEvent_t ev : pool->host_done)
+    if (ev) cudaEventDestroy(ev);
+  delete pool;
+}
 
 pace_status pace_pool_layout(const pace_pool* pool, int32_t head, size_t* record_offset,
                              size_t* record_bytes, size_t* slot_stride) {
@@ -239,6 +248,97 @@ pace_status pace_prefill(pace_pool* pool, int64_t T, const void* q, const void* 
                          const void* alpha, const void* beta, float* o, void* stream) {
   if (!pool) return PACE_ERR_INVALID_ARG;
   return pace_prefill_range(pool, 0, pool->dev.B, T, q, k, v, alpha, beta, o, stream);
+}
+
+namespace {
+struct HostSlot {   // byte offsets of one token's staging inside a slot
+  size_t q, k, v, a, b, o, bytes;
+};
+HostSlot host_slot(const pace_pool* pool) {
+  const size_t BH = (size_t)pool->dev.B * pool->dev.H;
+  const size_t esz = pool->dev.io == PACE_IO_BF16 ? 2 : 4;
+  HostSlot h;
+  h.q = 0;
+  h.k = round_up(BH * pool->dev.d_k * esz, 256);
+  h.v = h.k + round_up(BH * pool->dev.d_k * esz, 256);
+  h.a = h.v + round_up(BH * pool->dev.d_v * esz, 256);
+  h.b = h.a + round_up(BH * esz, 256);
+  h.o = h.b + round_up(BH * esz, 256);
+  h.bytes = h.o + round_up(BH * pool->dev.d_v * 4, 256);
+  return h;
+}
+}  // namespace
+
+pace_status pace_host_staging_bytes(const pace_pool* pool, size_t* bytes) {
+  if (!pool || !bytes) return PACE_ERR_INVALID_ARG;
+  *bytes = 2 * host_slot(pool).bytes;
+  return PACE_OK;
+}
+
+pace_status pace_decode_host(pace_pool* pool, int32_t n_tokens, const void* h_q, const void* h_k,
+                             const void* h_v, const void* h_alpha, const void* h_beta, float* h_o,
+                             void* d_staging, void* stream, void* h2d_stream, void* d2h_stream) {
+  if (!pool || n_tokens < 0 || !d_staging || !aligned(d_staging, 256)) return PACE_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!h_q || !h_k || !h_v || !h_alpha || !h_beta)) return PACE_ERR_INVALID_ARG;
+  const HostSlot hs = host_slot(pool);
+  const size_t BH = (size_t)pool->dev.B * pool->dev.H;
+  const size_t esz = pool->dev.io == PACE_IO_BF16 ? 2 : 4;
+  const size_t qb = BH * pool->dev.d_k * esz, vb = BH * pool->dev.d_v * esz, ab = BH * esz;
+  const size_t ob = BH * pool->dev.d_v * 4;
+  cudaStream_t cs = as_stream(stream), hs_in = as_stream(h2d_stream), hs_out = as_stream(d2h_stream);
+  if (cs == hs_in || cs == hs_out || hs_in == hs_out) return PACE_ERR_INVALID_ARG;
+  cudaError_t e = cudaSuccess;
+  cudaEvent_t* done = pool->host_done;   // [slot]: its last output copy (persists across calls)
+  for (int j = 0; j < 2 && e == cudaSuccess; ++j)
+    if (!done[j]) e = cudaEventCreateWithFlags(&done[j], cudaEventDisableTiming);
+  cudaEvent_t landed[2] = {nullptr, nullptr}, computed[2] = {nullptr, nullptr};
+  for (int j = 0; j < 2 && e == cudaSuccess; ++j) {
+    e = cudaEventCreateWithFlags(&landed[j], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&computed[j], cudaEventDisableTiming);
+  }
+  // The staging buffer of this pool's previous call is reused once each slot's
+  // last output copy is done, so consecutive calls keep the copy engines busy.
+  // A new buffer waits for all work already on `stream`.
+  const bool reuse = pool->host_staging == d_staging;
+  if (e == cudaSuccess && !reuse) {
+    for (int j = 0; j < 2 && e == cudaSuccess; ++j) e = cudaEventRecord(done[j], cs);
+    pool->host_staging = d_staging;
+  }
+  for (int t = 0; t < n_tokens && e == cudaSuccess; ++t) {
+    const int sl = t & 1;
+    uint8_t* base = static_cast<uint8_t*>(d_staging) + sl * hs.bytes;
+    const uint8_t* hq = static_cast<const uint8_t*>(h_q) + (size_t)t * qb;
+    const uint8_t* hk = static_cast<const uint8_t*>(h_k) + (size_t)t * qb;
+    const uint8_t* hv = static_cast<const uint8_t*>(h_v) + (size_t)t * vb;
+    const uint8_t* ha = static_cast<const uint8_t*>(h_alpha) + (size_t)t * ab;
+    const uint8_t* hb = static_cast<const uint8_t*>(h_beta) + (size_t)t * ab;
+    e = cudaStreamWaitEvent(hs_in, done[sl], 0);   // slot sl's previous token has been copied out
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.q, hq, qb, cudaMemcpyHostToDevice, hs_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.k, hk, qb, cudaMemcpyHostToDevice, hs_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.v, hv, vb, cudaMemcpyHostToDevice, hs_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.a, ha, ab, cudaMemcpyHostToDevice, hs_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.b, hb, ab, cudaMemcpyHostToDevice, hs_in);
+    if (e == cudaSuccess) e = cudaEventRecord(landed[sl], hs_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, landed[sl], 0);
+    if (e != cudaSuccess) break;
+    const pace::Span all{0, pool->dev.B, 0};
+    e = pace::launch_decode_step(pool->dev, all, base + hs.q, base + hs.k, base + hs.v, base + hs.a,
+                                 base + hs.b, reinterpret_cast<float*>(base + hs.o), cs);
+    if (e == cudaSuccess) e = pace::launch_commit(pool->dev, all, cs);   // heads whose buffer filled
+    if (e == cudaSuccess) e = cudaEventRecord(computed[sl], cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hs_out, computed[sl], 0);
+    if (e == cudaSuccess && h_o)
+      e = cudaMemcpyAsync(h_o + (size_t)t * BH * pool->dev.d_v, base + hs.o, ob, cudaMemcpyDeviceToHost, hs_out);
+    if (e == cudaSuccess) e = cudaEventRecord(done[sl], hs_out);
+  }
+  // `stream` completes after the last output copy
+  if (e == cudaSuccess && n_tokens > 0) e = cudaStreamWaitEvent(cs, done[(n_tokens - 1) & 1], 0);
+  if (e != cudaSuccess) pool->host_staging = nullptr;   // next call orders on `stream` again
+  for (int j = 0; j < 2; ++j) {
+    if (landed[j]) cudaEventDestroy(landed[j]);
+    if (computed[j]) cudaEventDestroy(computed[j]);
+  }
+  return from_cuda(e);
 }
 
 pace_status pace_commit_period(pace_pool* pool, void* stream) {

@@ -229,6 +229,33 @@ pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const 
                                float* o, int64_t n, int32_t d_k, int32_t d_v, void* stream);
 
 /*
+ * Decode from host memory.  n_tokens decode steps for every head with inputs
+ * and outputs in host memory (pinned for full copy speed):
+ *   h_q, h_k: [n_tokens][num_slots][num_heads][d_k], h_v: [...][d_v],
+ *   h_alpha, h_beta: [n_tokens][num_slots][num_heads] (io_dtype);
+ *   h_o: fp32 [n_tokens][num_slots][num_heads][d_v], or NULL.
+ * After every step each head whose buffer filled is committed (as
+ * pace_commit_period).  Token t's inputs are copied in on h2d_stream while
+ * token t-1 computes on `stream`, and its outputs are copied out on
+ * d2h_stream while token t+1 computes, through d_staging: a device buffer
+ * of pace_host_staging_bytes bytes (two token slots), 256-byte aligned,
+ * owned by the caller and not used by anything else meanwhile.  The first
+ * copies wait for the work already on `stream`, except when d_staging is the
+ * buffer of this pool's previous call: then each slot is refilled as soon as
+ * that call's last output copy from it is done, so consecutive calls keep
+ * the copy engines busy.  The three streams must be distinct
+ * (PACE_ERR_INVALID_ARG otherwise, as for a NULL or unaligned d_staging or a
+ * NULL input).  Enqueues only; `stream` completes after the last output
+ * copy.  Not safe to call concurrently on one pool.  This host-buffer entry
+ * point has no counterpart in the pages; it is the end-to-end path of a
+ * serving loop.
+ */
+pace_status pace_host_staging_bytes(const pace_pool* pool, size_t* bytes);
+pace_status pace_decode_host(pace_pool* pool, int32_t n_tokens, const void* h_q, const void* h_k,
+                             const void* h_v, const void* h_alpha, const void* h_beta, float* h_o,
+                             void* d_staging, void* stream, void* h2d_stream, void* d2h_stream);
+
+/*
  * Chunked fp32 prefill (the chunked prefill kernels that [P2] "Periodic
  * Rounding" cites; [P4] flowchart "State update, chunked, high precision").
  * For every head of the slots (all of them, or [slot_begin, slot_begin +
