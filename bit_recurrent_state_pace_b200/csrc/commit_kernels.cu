@@ -82,9 +82,8 @@ struct alignas(16) Smem {
   WarpTab<D> wt[C::RB];
   uint64_t bar[3];
   int hq[3];                                      // head staged in each slot
-  float xinv;
   int next_head;
-  int slow;
+  int slow[2];                                    // by head parity: exact-encode fallback needed
 };
 
 // First head index >= from (stepping by step, below end) with a full buffer.
@@ -144,9 +143,11 @@ __device__ __forceinline__ void load_rows_smem(RowBlock<D, BITS>& rb, const uint
 
 // EXACT: the pool's period equals PMAX, so every loop bound over tokens is a
 // compile-time constant.
+// Returns false (every thread) when the staged copies of this head did not
+// arrive in time (ok == false in some thread); nothing is written then.
 template <int D, bool BF16, int PMAX, int BITS, bool EXACT, class Issue>
-__device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot,
-                            Issue&& issue_next) {
+__device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot,
+                            bool ok, int parity_bit, Issue&& issue_next) {
   using C = Cfg<D, BF16, PMAX>;
   constexpr int KS = C::KS, NT = C::NT, NTX = C::NTX, KU = C::KU, NU = C::NU;
   constexpr int ROWB = D * BITS / 8;
@@ -168,14 +169,15 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   const float* W = s_gr;
   const float* gam = s_gr + P * P;
   const float gP = gam[P - 1];
+  // (the operands of the previous head were last read before its absmax
+  // barrier, so these tables are rebuilt without a barrier of their own)
   for (int j = tid; j < D; j += C::THREADS) sm.sc[j] = __half2float(__ushort_as_half(s_sc[j]));
   // one power-of-two normalisation of the X operand for the whole head
   const float bmax = col ? s_gr[P * P + P] * s_gr[P * P + P + 1] : s_gr[P * P + P];
   int exx = 0;
   if (bmax >= 1.17549435e-38f && bmax < INFINITY) exx = max(-120, min(120, 14 - exp2_floor(bmax)));
   const float upx = pow2i(exx);
-  if (tid == 0) sm.xinv = pow2i(-exx);
-  __syncthreads();   // sm.sc
+  const float xinv = pow2i(-exx);
   {
     // X operand, built by fragment owner: entry (x, ks, g, t) holds rows
     // k = 2t, 2t+1 | 2t+8, 2t+9 (key channels jof(t, ks, 0..3)) of column
@@ -192,7 +194,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
         for (int pos = 0; pos < 4; ++pos) {
           const int j = jof<D, BITS>(tt, ks, pos);
           const float kv = io_at(s_kv + s * C::ROWS, j, BF16);
-          const float xv = (col ? kv * sm.sc[j] : kv) * upx;
+          const float xv = (col ? kv * __half2float(__ushort_as_half(s_sc[j])) : kv) * upx;
           hv[pos] = __float2half_rn(xv);
           lv[pos] = __float2half_rn(xv - __half2float(hv[pos]));
         }
@@ -235,7 +237,10 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       sm.bkf[tau][u][gg][tt] = make_uint2(wv[0], wv[1]);
     }
   }
-  __syncthreads();
+  if (__syncthreads_or(!ok)) return false;
+  // every thread is past the previous head's encode: its flag is free for the head after this one
+  if (tid == 0) sm.slow[parity_bit ^ 1] = 0;
+  int& slow_flag = sm.slow[parity_bit];
 
   // ---- phase 2: this warp's 16 rows ------------------------------------------
   const int i0 = 16 * w + g, i1 = i0 + 8;
@@ -261,7 +266,6 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   float r[PMAX][2];
   {
     float ro[NTX][2];
-    const float xinv = sm.xinv;
     const float s0 = (col ? 1.f : sm.sc[i0]) * xinv, s1 = (col ? 1.f : sm.sc[i1]) * xinv;
 #pragma unroll
     for (int x = 0; x < NTX; ++x) {
@@ -444,7 +448,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       sm.qf[i1] = s1.sf > 0.f ? __frcp_rn(s1.sf) : 0.f;
       sm.sfv[i0] = s0.sf;
       sm.sfv[i1] = s1.sf;
-      if (bad) sm.slow = 1;
+      if (bad) slow_flag = 1;
     }
   }
   __syncthreads();
@@ -458,13 +462,13 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       rsc[j] = s.bits;
       sm.qf[j] = s.sf > 0.f ? __frcp_rn(s.sf) : 0.f;
       sm.sfv[j] = s.sf;
-      if (!isfinite(a) || (s.bits == 0x7BFF && a / qmax > 65504.f)) sm.slow = 1;
+      if (!isfinite(a) || (s.bits == 0x7BFF && a / qmax > 65504.f)) slow_flag = 1;
     }
     __syncthreads();
   }
 
   // ---- encode and store this warp's rows ------------------------------------
-  const bool slow = sm.slow != 0;
+  const bool slow = slow_flag != 0;
   if (col) {
     for (int e = lane; e < KS * 4; e += 32) {
       const int ks = e >> 2, tt = e & 3;
@@ -537,6 +541,7 @@ __device__ void commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   if (!slow) encode_rows(std::true_type{});
   else encode_rows(std::false_type{});
   if (tid == 0) p.fill[head] = 0;
+  return true;
 }
 
 template <int D, bool BF16, int PMAX, bool EXACT>
@@ -568,23 +573,15 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     cand = h;
     if (cand < n_heads) cand_fill = p.fill[cand];
   }
-  if (tid == 0) sm.slow = 0;
+  if (tid == 0) sm.slow[0] = sm.slow[1] = 0;
   __syncthreads();
   uint32_t parity = 0u;
-  int s = 0;
+  int s = 0, iter = 0;
   while (true) {
     const int head = sm.hq[s];
     if (head >= n_heads) break;
     const bool ok = mbar_wait_bounded(&sm.bar[s], (parity >> s) & 1u, p.flags);
     parity ^= 1u << s;
-    if (__syncthreads_or(!ok)) {
-      if (tid == ISS)
-        for (int i = 0; i < 3; ++i)
-          if (i != s && sm.hq[i] < n_heads) mbar_wait_bounded(&sm.bar[i], (parity >> i) & 1u, nullptr);
-      __syncthreads();
-      return;
-    }
-    if (tid == 0) sm.slow = 0;   // every thread is past the previous head's encode
     const int s2 = s == 0 ? 2 : s - 1;   // slot of the head two ahead (held the previous head)
     auto issue_next = [&]() {
       if (tid == ISS) {
@@ -596,10 +593,18 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
         if (cand < n_heads) cand_fill = p.fill[cand];
       }
     };
-    if (p.bits[head % p.H] == 4)
-      commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s], issue_next);
-    else
-      commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s], issue_next);
+    const bool done =
+        p.bits[head % p.H] == 4
+            ? commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s], ok, iter & 1, issue_next)
+            : commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s], ok, iter & 1, issue_next);
+    if (!done) {   // a bounded wait gave up: let the copies in flight land, then leave
+      if (tid == ISS)
+        for (int i = 0; i < 3; ++i)
+          if (i != s && sm.hq[i] < n_heads) mbar_wait_bounded(&sm.bar[i], (parity >> i) & 1u, nullptr);
+      __syncthreads();
+      return;
+    }
+    ++iter;
     s = s == 2 ? 0 : s + 1;
   }
 }
