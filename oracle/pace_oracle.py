@@ -44,6 +44,14 @@ Pages cited (by title and section):
    per-head bit widths, handled by calling ``quantize`` with bits 4 or 8.
    ``decay_rates`` / ``select_head_bits`` choose the 8-bit heads from the
    gates (mean -ln alpha per head, the slowest-decaying heads first).
+6. Adaptive period.  [P4] "Research angle": round when the accumulated
+   update norm crosses a threshold rather than every k tokens.  Reading: the
+   accumulated update after n buffered tokens is what the writes added to
+   the decayed stored state, ``Delta_n = S_n - gamma_n S~0`` (a pure decay is
+   a rescaling that needs no re-encoding), in the Frobenius norm; a head is
+   rounded after token n when ``||Delta_n||_F >= tau`` and in any case when
+   its buffer of P tokens is full.  ``update_norm2`` writes the definition
+   out; ``pace_run_adaptive`` is the per-head driver.
 
 Everything here is fp64 except the quantiser, which takes the fp32 state and
 reproduces the fp32/fp16 operations of the encoding one by one with numpy's
@@ -408,3 +416,64 @@ def select_head_bits(rates, num_int8: int) -> List[int]:
     for h in order[:num_int8]:
         bits[h] = 8
     return bits
+
+
+# --------------------------------------------------------------------------
+# Adaptive period, [P4] "Research angle": a head is rounded when its
+# accumulated update crosses a threshold instead of after a fixed number of
+# tokens; the buffer's capacity P still bounds the period.
+# --------------------------------------------------------------------------
+
+def update_norm2(S_n, S0, gamma_n) -> np.ndarray:
+    """||S_n - gamma_n S0||_F^2 per head (fp64): the squared Frobenius norm of
+    what the writes since the last rounding added to the decayed state.
+    S_n, S0 [N, d_v, d_k]; gamma_n [N] (product of the period's alphas)."""
+    S_n = np.asarray(S_n, dtype=np.float64)
+    S0 = np.asarray(S0, dtype=np.float64)
+    g = np.asarray(gamma_n, dtype=np.float64)[:, None, None]
+    delta = S_n - g * S0
+    return np.sum(delta * delta, axis=(1, 2))
+
+
+def pace_run_adaptive(state: PoolState, tokens: Sequence[Dict[str, np.ndarray]], P: int,
+                      tau: float, step=gdn_step):
+    """Decode ``tokens`` with a per-head adaptive period, every head starting
+    at a period boundary.
+
+    After each token every head advances its fp64 working state exactly from
+    its dequantised stored state; head h is rounded (fp32, then its own bit
+    width) when it holds P tokens or when update_norm2 >= tau^2, and restarts
+    from its newly stored state.  tau = inf gives the fixed period P; tau = 0
+    rounds after every token.
+
+    Returns (outputs per token [N, d_v], final PoolState, rounded [T][N] bool,
+    norm2 [T][N] (before any rounding of that token), flags).
+    """
+    S0 = state.dequantized()
+    S = S0.copy()
+    N = S.shape[0]
+    codes = list(state.codes)
+    scales = list(state.scales)
+    gamma = np.ones(N)
+    n = np.zeros(N, dtype=np.int64)
+    tau2 = float(tau) * float(tau)
+    outs, rounded, norms, flags = [], [], [], 0
+    for tok in tokens:
+        S, o = step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
+        outs.append(o)
+        gamma = gamma * np.asarray(tok["alpha"], dtype=np.float64)
+        n += 1
+        norm2 = update_norm2(S, S0, gamma)
+        due = (n == P) | (norm2 >= tau2)
+        for i in np.nonzero(due)[0]:
+            c, sc, f = quantize(S[i:i + 1].astype(np.float32), state.bits[i], state.axis)
+            flags |= f
+            codes[i], scales[i] = c[0], sc[0]
+            S0[i] = dequantize(c[0], sc[0], state.axis)
+            S[i] = S0[i]
+            gamma[i] = 1.0
+            n[i] = 0
+        rounded.append(due)
+        norms.append(norm2)
+    final = PoolState(codes, scales, state.bits, state.axis)
+    return outs, final, rounded, norms, flags

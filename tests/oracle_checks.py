@@ -427,3 +427,127 @@ def check_step_forms_agree(gdn_step, gdn_step_delta, seed=0):
         S2, o2 = gdn_step_delta(S, tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"])
         assert np.allclose(S1, S2, rtol=1e-13, atol=1e-13) and np.allclose(o1, o2, rtol=1e-13, atol=1e-13)
         S = S1
+
+
+# ---------------- adaptive period ----------------
+
+def _random_pool_state(rng, N, d_v, d_k, bits, axis, quantize):
+    S = (rng.standard_normal((N, d_v, d_k)) * 0.5).astype(np.float32)
+    codes, scales = [], []
+    for i in range(N):
+        c, s, _ = quantize(S[i:i + 1], bits[i], axis)
+        codes.append(c[0])
+        scales.append(s[0])
+    return codes, scales
+
+
+def check_update_norm_closed_forms(update_norm2, gdn_step, seed=0):
+    """||S_n - gamma_n S0||_F^2 against what the recurrence fixes: zero without
+    writes, the rank-1 norm after one token, and the one-token recursion
+    N_n = a^2 N_{n-1} + 2 a u.(Delta_{n-1} k) + |u|^2 |k|^2 with
+    u = b (v - a S_{n-1} k), which follows from S_n = a S_{n-1} + u k^T."""
+    rng = np.random.default_rng(seed)
+    N, d_v, d_k = 5, 9, 7
+    S0 = rng.standard_normal((N, d_v, d_k))
+    # no writes (beta = 0): the state only decays
+    S, g = S0, np.ones(N)
+    for tk in random_tokens(rng, N, 4, d_k, d_v):
+        S, _ = gdn_step(S, tk["q"], tk["k"], tk["v"], tk["alpha"], np.zeros(N))
+        g = g * tk["alpha"]
+        assert np.all(update_norm2(S, S0, g) <= 1e-26 * np.sum(S0 * S0, axis=(1, 2)))
+    # one token: Delta_1 = b (v - a S0 k) k^T, a rank-1 matrix
+    tk = random_tokens(rng, N, 1, d_k, d_v)[0]
+    k = tk["k"] * rng.uniform(0.5, 2.0, (N, 1))
+    S1, _ = gdn_step(S0, tk["q"], k, tk["v"], tk["alpha"], tk["beta"])
+    err = tk["v"] - tk["alpha"][:, None] * np.einsum("nij,nj->ni", S0, k)
+    ref = tk["beta"] ** 2 * np.sum(err * err, axis=1) * np.sum(k * k, axis=1)
+    got = update_norm2(S1, S0, tk["alpha"])
+    assert np.allclose(got, ref, rtol=1e-12, atol=0), (got, ref)
+    # the recursion over several tokens
+    S, g, prev = S0, np.ones(N), np.zeros(N)
+    for tk in random_tokens(rng, N, 6, d_k, d_v):
+        a, b = tk["alpha"], tk["beta"]
+        Sk = np.einsum("nij,nj->ni", S, tk["k"])
+        delta_k = Sk - g[:, None] * np.einsum("nij,nj->ni", S0, tk["k"])
+        u = b[:, None] * (tk["v"] - a[:, None] * Sk)
+        rec = a * a * prev + 2 * a * np.sum(u * delta_k, 1) + np.sum(u * u, 1) * np.sum(tk["k"] ** 2, 1)
+        S, _ = gdn_step(S, tk["q"], tk["k"], tk["v"], a, b)
+        g = g * a
+        got = update_norm2(S, S0, g)
+        assert np.allclose(got, rec, rtol=1e-10, atol=0), (got, rec)
+        prev = got
+
+
+def check_adaptive_limits(pace_run_adaptive, pace_run, per_token_rounding, PoolState, quantize,
+                          seed=0):
+    """tau = inf is the fixed period P; tau = 0 rounds after every token."""
+    rng = np.random.default_rng(seed)
+    N, d_v, d_k, P = 6, 8, 8, 4
+    bits = [4, 8, 4, 4, 8, 4]
+    for axis in ("col", "row"):
+        codes, scales = _random_pool_state(rng, N, d_v, d_k, bits, axis, quantize)
+        st = PoolState(codes, scales, bits, axis)
+        toks = random_tokens(rng, N, 11, d_k, d_v)
+        o_a, fin_a, rounded, _, _ = pace_run_adaptive(st, toks, P, float("inf"))
+        o_f, fin_f, _, _, _ = pace_run(st, toks, P)
+        for x, y in zip(o_a, o_f):
+            assert np.array_equal(x, y)
+        assert all(np.array_equal(a, b) for a, b in zip(fin_a.codes, fin_f.codes))
+        assert [bool(r.all()) for r in rounded] == [(t + 1) % P == 0 for t in range(len(toks))]
+        o_a, fin_a, rounded, _, _ = pace_run_adaptive(st, toks, P, 0.0)
+        o_p, fin_p = per_token_rounding(st, toks)
+        for x, y in zip(o_a, o_p):
+            assert np.array_equal(x, y)
+        assert all(np.array_equal(a, b) for a, b in zip(fin_a.codes, fin_p.codes))
+        assert all(r.all() for r in rounded)
+        # a pure decay has a zero update, which still reaches tau = 0
+        still = [dict(tk, beta=np.zeros(N)) for tk in toks]
+        _, _, rounded, norms, _ = pace_run_adaptive(st, still, P, 0.0)
+        assert all(r.all() for r in rounded) and all(np.all(x == 0.0) for x in norms)
+
+
+def check_adaptive_driver_per_head(pace_run_adaptive, chunk_form, PoolState, quantize, dequantize,
+                                   seed=0):
+    """A finite threshold, replayed head by head in chunk form: each head keeps
+    its own buffer, its state after n tokens and the accumulated update
+    sum_s gamma_{n/s} u_s k_s^T both come from chunk_form, and it is rounded
+    when the update's squared norm reaches tau^2 or the buffer holds P."""
+    rng = np.random.default_rng(seed)
+    N, d_v, d_k, P, T, tau = 6, 8, 8, 5, 24, 2.0
+    bits = [4, 4, 8, 4, 8, 4]
+    axis = "col"
+    codes, scales = _random_pool_state(rng, N, d_v, d_k, bits, axis, quantize)
+    st = PoolState(codes, scales, bits, axis)
+    toks = random_tokens(rng, N, T, d_k, d_v)
+    o_a, fin_a, rounded, norms, _ = pace_run_adaptive(st, toks, P, tau)
+    n_rounded = 0
+    for i in range(N):
+        c, s = codes[i], scales[i]
+        buf = []
+        for t, tk in enumerate(toks):
+            buf.append({key: np.asarray(val)[i:i + 1] for key, val in tk.items()})
+            S0 = dequantize(c, s, axis).astype(np.float64)[None]
+            K = np.stack([b["k"] for b in buf], 1)
+            V = np.stack([b["v"] for b in buf], 1)
+            A = np.stack([b["alpha"] for b in buf], 1)
+            B = np.stack([b["beta"] for b in buf], 1)
+            S_n, U, o = chunk_form(S0, K, V, A, B, buf[-1]["q"])
+            n = len(buf)
+            g = np.array([np.prod(A[0, s + 1:]) for s in range(n)])   # gamma_{n/s}
+            delta = np.einsum("s,si,sj->ij", g, U[0], K[0])
+            norm2 = float(np.sum(delta * delta))
+            assert abs(norm2 - tau * tau) > 1e-9 * tau * tau, "tie: choose another seed"
+            assert np.allclose(norms[t][i], norm2, rtol=1e-9), (i, t)
+            assert np.allclose(o_a[t][i], o[0], rtol=1e-10, atol=1e-12), (i, t)
+            due = n == P or norm2 >= tau * tau
+            assert bool(rounded[t][i]) == due, (i, t)
+            if due:
+                n_rounded += 1
+                c2, s2, _ = quantize(S_n.astype(np.float32), bits[i], axis)
+                c, s = c2[0], s2[0]
+                buf = []
+        assert np.array_equal(fin_a.codes[i], c) and np.array_equal(
+            fin_a.scales[i].view(np.uint16), np.asarray(s).view(np.uint16)), i
+    # the threshold, not the buffer, must end most periods here
+    full = sum(bool(r[i]) for r in rounded for i in range(N))
+    assert n_rounded == full and full > N * T // P

@@ -169,3 +169,83 @@ def test_pack_mutant_is_caught():
         hi = codes[..., 0::2].astype(np.int16) & 0xF
         return (lo | (hi << 4)).astype(np.uint8)
     assert _fails(ck.check_encoder_golden, orc.quantize, pack_swapped)
+
+
+# ---------------- adaptive-period mutants ----------------
+
+def _norm_factory(kind):
+    def update_norm2(S_n, S0, gamma_n):
+        S_n = np.asarray(S_n, dtype=np.float64)
+        S0 = np.asarray(S0, dtype=np.float64)
+        g = np.asarray(gamma_n, dtype=np.float64)[:, None, None]
+        if kind == "no_gamma":
+            g = np.ones_like(g)
+        if kind == "gamma_squared":
+            g = g * g
+        delta = S_n - g * S0
+        if kind == "max_not_sum":
+            return np.max(delta * delta, axis=(1, 2))
+        r = np.sum(delta * delta, axis=(1, 2))
+        return np.sqrt(r) if kind == "not_squared" else r
+    return update_norm2
+
+
+NORM_MUTANTS = ["no_gamma", "gamma_squared", "max_not_sum", "not_squared"]
+
+
+@pytest.mark.parametrize("kind", NORM_MUTANTS + ["none"])
+def test_update_norm_mutant_is_caught(kind):
+    caught = _fails(ck.check_update_norm_closed_forms, _norm_factory(kind), orc.gdn_step)
+    assert caught == (kind != "none"), kind
+
+
+def _adaptive_factory(kind):
+    def run(state, tokens, P, tau, step=orc.gdn_step):
+        S0 = state.dequantized()
+        S = S0.copy()
+        N = S.shape[0]
+        codes, scales = list(state.codes), list(state.scales)
+        gamma, n = np.ones(N), np.zeros(N, dtype=np.int64)
+        tau2 = float(tau) * float(tau)
+        outs, rounded, norms = [], [], []
+        for tok in tokens:
+            S, o = step(S, tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
+            outs.append(o)
+            gamma = gamma * np.asarray(tok["alpha"], dtype=np.float64)
+            n += 1
+            norm2 = orc.update_norm2(S, S0, gamma)
+            if kind == "strict":
+                due = (n == P) | (norm2 > tau2)
+            elif kind == "period_off_by_one":
+                due = (n == P + 1) | (norm2 >= tau2)
+            elif kind == "norm_not_squared_threshold":
+                due = (n == P) | (norm2 >= float(tau))
+            else:
+                due = (n == P) | (norm2 >= tau2)
+            for i in np.nonzero(due)[0]:
+                c, sc, _ = orc.quantize(S[i:i + 1].astype(np.float32), state.bits[i], state.axis)
+                codes[i], scales[i] = c[0], sc[0]
+                S0[i] = orc.dequantize(c[0], sc[0], state.axis)
+                if kind != "no_restart":
+                    S[i] = S0[i]
+                if kind != "no_gamma_reset":
+                    gamma[i] = 1.0
+                n[i] = 0
+            rounded.append(due)
+            norms.append(norm2)
+        return outs, orc.PoolState(codes, scales, state.bits, state.axis), rounded, norms, 0
+    return run
+
+
+ADAPTIVE_MUTANTS = ["strict", "period_off_by_one", "norm_not_squared_threshold", "no_restart",
+                    "no_gamma_reset"]
+
+
+@pytest.mark.parametrize("kind", ADAPTIVE_MUTANTS + ["none"])
+def test_adaptive_driver_mutant_is_caught(kind):
+    run = _adaptive_factory(kind)
+    caught = (_fails(ck.check_adaptive_limits, run, orc.pace_run, orc.per_token_rounding,
+                     orc.PoolState, orc.quantize)
+              or _fails(ck.check_adaptive_driver_per_head, run, orc.chunk_form, orc.PoolState,
+                        orc.quantize, orc.dequantize))
+    assert caught == (kind != "none"), kind

@@ -131,3 +131,17 @@ def test_relative_error_metric():
     assert orc.relative_error(ref, ref)[0] == 0
     assert orc.relative_error(ref + np.array([[0, 0.004, 0]]), ref)[0] == pytest.approx(0.002)
     assert orc.relative_error(np.zeros((1, 3)), np.zeros((1, 3)))[0] == 0
+
+
+def test_update_norm_closed_forms():
+    ck.check_update_norm_closed_forms(orc.update_norm2, orc.gdn_step)
+
+
+def test_adaptive_period_limits():
+    ck.check_adaptive_limits(orc.pace_run_adaptive, orc.pace_run, orc.per_token_rounding,
+                             orc.PoolState, orc.quantize)
+
+
+def test_adaptive_period_replayed_per_head_in_chunk_form():
+    ck.check_adaptive_driver_per_head(orc.pace_run_adaptive, orc.chunk_form, orc.PoolState,
+                                      orc.quantize, orc.dequantize)
