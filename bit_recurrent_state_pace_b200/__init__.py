@@ -21,11 +21,12 @@ __all__ = [
     "PaceError", "lib", "LIB_PATH",
     "PACE_SCALE_COL", "PACE_SCALE_ROW", "PACE_IO_BF16", "PACE_IO_F32",
     "PACE_FLAG_NONFINITE", "PACE_FLAG_SCALE_OVERFLOW", "PACE_FLAG_BUFFER_FULL", "PACE_FLAG_TIMEOUT",
+    "PACE_FILL_COMMIT",
     "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
     "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
     "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
     "pace_select_head_bits", "pace_prefill", "pace_prefill_range", "pace_host_staging_bytes",
-    "pace_decode_host",
+    "pace_decode_host", "pace_set_commit_threshold",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -39,6 +40,7 @@ PACE_FLAG_NONFINITE = 0x1
 PACE_FLAG_SCALE_OVERFLOW = 0x2
 PACE_FLAG_BUFFER_FULL = 0x4
 PACE_FLAG_TIMEOUT = 0x8
+PACE_FILL_COMMIT = 0x100
 PACE_OK, PACE_ERR_DEVICE_FLAGS = 0, 4
 
 
@@ -77,6 +79,7 @@ def _load():
         "pace_decay_rates": [P, I64, I32, I32, P, P],
         "pace_prefill": [P, I64, P, P, P, P, P, F32p, P],
         "pace_host_staging_bytes": [P, Sp],
+        "pace_set_commit_threshold": [P, ctypes.c_float],
         "pace_decode_host": [P, I32, P, P, P, P, P, P, P, P, P, P],
         "pace_prefill_range": [P, I32, I32, I64, P, P, P, P, P, F32p, P],
         "pace_select_head_bits": [P, I32, I32, P],
@@ -182,6 +185,10 @@ def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
 
 def pace_commit_period(handle: int, stream=None) -> None:
     _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_set_commit_threshold(handle: int, tau: float) -> None:
+    _check("pace_set_commit_threshold", lib.pace_set_commit_threshold(handle, float(tau)))
 
 
 def pace_host_staging_bytes(handle: int) -> int:
@@ -365,6 +372,11 @@ class PacePool:
         """T tokens [T][B][H][d] through the chunked fp32 prefill; returns o."""
         pace_prefill(self.handle, int(q.shape[0]), q, k, v, alpha, beta, o, stream)
         return o
+
+    def set_commit_threshold(self, tau: float) -> None:
+        """Adaptive period: a head is committed early once the Frobenius norm of
+        its update since the last rounding reaches tau (inf: fixed period)."""
+        pace_set_commit_threshold(self.handle, tau)
 
     def decode_host(self, q, k, v, alpha, beta, o=None, stream=None) -> None:
         """T decode steps (each followed by the commit of full heads) from host

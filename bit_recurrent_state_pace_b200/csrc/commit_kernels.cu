@@ -82,14 +82,15 @@ struct alignas(16) Smem {
   WarpTab<D> wt[C::RB];
   uint64_t bar[3];
   int hq[3];                                      // head staged in each slot
+  int hn[3];                                      // its buffered tokens
   int next_head;
   int slow[2];                                    // by head parity: exact-encode fallback needed
 };
 
-// First head index >= from (stepping by step, below end) with a full buffer.
+// First head index >= from (stepping by step, below end) due for a commit.
 __device__ __forceinline__ int find_full(const PoolDev& p, int from, int step, int end) {
   int hd = from;
-  while (hd < end && p.fill[hd] != p.P) hd += step;
+  while (hd < end && !commit_due(p.fill[hd], p.P)) hd += step;
   return hd;
 }
 
@@ -145,14 +146,16 @@ __device__ __forceinline__ void load_rows_smem(RowBlock<D, BITS>& rb, const uint
 // compile-time constant.
 // Returns false (every thread) when the staged copies of this head did not
 // arrive in time (ok == false in some thread); nothing is written then.
+// n_tok: the head's buffered tokens (P, or fewer for a head marked early).
 template <int D, bool BF16, int PMAX, int BITS, bool EXACT, class Issue>
 __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot,
-                            bool ok, int parity_bit, Issue&& issue_next) {
+                            int n_tok, bool ok, int parity_bit, Issue&& issue_next) {
   using C = Cfg<D, BF16, PMAX>;
   constexpr int KS = C::KS, NT = C::NT, NTX = C::NTX, KU = C::KU, NU = C::NU;
   constexpr int ROWB = D * BITS / 8;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
-  const int P = EXACT ? PMAX : p.P, h = head % p.H, b = head / p.H;
+  // P: tokens to apply; PS: the pool's period, the stride of the factor block
+  const int P = EXACT ? PMAX : n_tok, PS = EXACT ? PMAX : p.P, h = head % p.H, b = head / p.H;
   const bool col = p.axis == PACE_SCALE_COL;
   const int qmax = BITS == 4 ? 7 : 127;
   uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
@@ -167,13 +170,13 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   // W[s][s'] (P x P), gamma_s (P), max |k| and the largest stored scale were
   // left in the Gram block by the decode step that buffered the P-th token.
   const float* W = s_gr;
-  const float* gam = s_gr + P * P;
+  const float* gam = s_gr + PS * PS;
   const float gP = gam[P - 1];
   // (the operands of the previous head were last read before its absmax
   // barrier, so these tables are rebuilt without a barrier of their own)
   for (int j = tid; j < D; j += C::THREADS) sm.sc[j] = __half2float(__ushort_as_half(s_sc[j]));
   // one power-of-two normalisation of the X operand for the whole head
-  const float bmax = col ? s_gr[P * P + P] * s_gr[P * P + P + 1] : s_gr[P * P + P];
+  const float bmax = col ? s_gr[PS * PS + PS] * s_gr[PS * PS + PS + 1] : s_gr[PS * PS + PS];
   int exx = 0;
   if (bmax >= 1.17549435e-38f && bmax < INFINITY) exx = max(-120, min(120, 14 - exp2_floor(bmax)));
   const float upx = pow2i(exx);
@@ -297,16 +300,16 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   for (int q = 0; q < NU; ++q) {
     const int s = (2 * t + (q & 1) + 8 * (q >> 1)) % PMAX;
     float wrow[PMAX];
-    if ((P & 3) == 0 && s < P) {          // row s of W in 16-byte pieces
+    if ((PS & 3) == 0 && s < P) {         // row s of W in 16-byte pieces (zero beyond P)
 #pragma unroll
       for (int c = 0; c < PMAX / 4; ++c) {
-        const float4 w4 = 4 * c < P ? reinterpret_cast<const float4*>(W + s * P)[c]
+        const float4 w4 = 4 * c < P ? reinterpret_cast<const float4*>(W + s * PS)[c]
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
         wrow[4 * c] = w4.x; wrow[4 * c + 1] = w4.y; wrow[4 * c + 2] = w4.z; wrow[4 * c + 3] = w4.w;
       }
     } else {
 #pragma unroll
-      for (int sp = 0; sp < PMAX; ++sp) wrow[sp] = (s < P && sp < P) ? W[s * P + sp] : 0.f;
+      for (int sp = 0; sp < PMAX; ++sp) wrow[sp] = (s < P && sp < P) ? W[s * PS + sp] : 0.f;
     }
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
@@ -566,6 +569,7 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     for (int i = 0; i < 2; ++i) {
       sm.hq[i] = h;
       if (h < n_heads) {
+        sm.hn[i] = p.fill[h] & 0xff;
         issue_head<D, BF16, PMAX>(p, h, sm, i);
         h = find_full(p, h + gridDim.x, gridDim.x, n_heads);
       }
@@ -586,17 +590,23 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     auto issue_next = [&]() {
       if (tid == ISS) {
         int nxt = cand;
-        if (nxt < n_heads && cand_fill != p.P) nxt = find_full(p, nxt + gridDim.x, gridDim.x, n_heads);
+        if (nxt < n_heads && !commit_due(cand_fill, p.P))
+          nxt = find_full(p, nxt + gridDim.x, gridDim.x, n_heads);
         sm.hq[s2] = nxt;
-        if (nxt < n_heads) issue_head<D, BF16, PMAX>(p, nxt, sm, s2);
+        if (nxt < n_heads) {
+          sm.hn[s2] = (nxt == cand ? cand_fill : p.fill[nxt]) & 0xff;
+          issue_head<D, BF16, PMAX>(p, nxt, sm, s2);
+        }
         cand = nxt < n_heads ? nxt + gridDim.x : n_heads;
         if (cand < n_heads) cand_fill = p.fill[cand];
       }
     };
     const bool done =
         p.bits[head % p.H] == 4
-            ? commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s], ok, iter & 1, issue_next)
-            : commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s], ok, iter & 1, issue_next);
+            ? commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s], sm.hn[s], ok, iter & 1,
+                                                   issue_next)
+            : commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s], sm.hn[s], ok, iter & 1,
+                                                   issue_next);
     if (!done) {   // a bounded wait gave up: let the copies in flight land, then leave
       if (tid == ISS)
         for (int i = 0; i < 3; ++i)
@@ -640,7 +650,8 @@ cudaError_t launch_t(const PoolDev& p, const Span& sp, cudaStream_t st) {
 
 template <int D, bool BF16>
 cudaError_t launch_p(const PoolDev& p, const Span& sp, cudaStream_t st) {
-  switch (p.P) {
+  // heads marked early hold fewer than P tokens: per-head token counts
+  if (!p.adaptive) switch (p.P) {
     case 4: return launch_t<D, BF16, 4, true>(p, sp, st);
     case 8: return launch_t<D, BF16, 8, true>(p, sp, st);
     case 16: return launch_t<D, BF16, 16, true>(p, sp, st);

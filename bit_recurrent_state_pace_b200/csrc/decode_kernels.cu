@@ -43,13 +43,106 @@ constexpr int kWarpsPerBlock = 8;
 constexpr int kThreads = kWarpsPerBlock * 32;
 constexpr unsigned FULL = 0xffffffffu;
 
-template <int D>
+// ADAPT (commit threshold set): two more right-hand sides, a^ and b^ (digit
+// rows 4..6 and 8..10), for the accumulated-update norm.
+template <int D, bool ADAPT>
 struct alignas(16) WarpScratch {
-  uint8_t dig[4][D];               // digits 0..2 of the right-hand side, row 3 = zeros
+  static constexpr int NDIG = ADAPT ? 11 : 4;
+  uint8_t dig[NDIG][D];            // digits 0..2 of q^ (row 3 = zeros), then of a^, b^
   float y[D];                      // S~0 q^ by row, before the row scale
+  float ya[ADAPT ? D : 1];         // S~0 a^
+  float yb[ADAPT ? D : 1];         // S~0 b^
   float A[PACE_MAX_PERIOD * PACE_MAX_PERIOD];   // period end: A[t][s]
   float gsb[3][PACE_MAX_PERIOD];                // period end: gamma_s, gamma_{P/s}, beta_s
 };
+
+// Right-hand side x (the lane's EPL key channels, times the column scales)
+// as 22-bit fixed point, split into three balanced base-256 digits:
+// x 2^e = d0 + 256 d1 + 65536 d2.  Writes digit rows dig[0..2] in the
+// order the code fragments expect and returns 2^-e; dsum: the lane's digit
+// sums (for the offset-byte correction of INT4 codes).
+template <int D, int EPL, int BITS>
+__device__ __forceinline__ float rhs_digits(const float (&x)[EPL], uint8_t (*dig)[D], int lane,
+                                            int (&dsum)[3]) {
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+  int ex = 0;
+  if (m > 0.f && m < INFINITY) ex = max(-120, min(120, 21 - ilogbf(m)));
+  const float up = ldexpf(1.f, ex);
+  dsum[0] = dsum[1] = dsum[2] = 0;
+  uint32_t dw[3] = {0u, 0u, 0u};    // digit bytes of this lane's EPL elements
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int Q = __float2int_rn(x[e] * up);
+    const int d0 = (int)(int8_t)(Q & 0xff);
+    const int r1 = (Q - d0) >> 8;
+    const int d1 = (int)(int8_t)(r1 & 0xff);
+    const int d2 = (r1 - d1) >> 8;
+    dsum[0] += d0; dsum[1] += d1; dsum[2] += d2;
+    dw[0] |= (uint32_t)(d0 & 0xff) << (8 * e);
+    dw[1] |= (uint32_t)(d1 & 0xff) << (8 * e);
+    dw[2] |= (uint32_t)(d2 & 0xff) << (8 * e);
+  }
+  if (BITS == 8) {
+    // natural key-channel order
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+      uint8_t* dst = &dig[d][EPL * lane];
+      if (EPL == 4) *reinterpret_cast<uint32_t*>(dst) = dw[d];
+      else if (EPL == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)dw[d];
+      else *dst = (uint8_t)dw[d];
+    }
+  } else {
+    // within each group of 8 key channels: even offsets first, then odd
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int j = EPL * lane + e, o = j & 7;
+      const int at = (j & ~7) + ((o & 1) ? 4 + (o >> 1) : (o >> 1));
+#pragma unroll
+      for (int d = 0; d < 3; ++d) dig[d][at] = (uint8_t)(dw[d] >> (8 * e));
+    }
+  }
+  return ldexpf(1.f, -ex);
+}
+
+// INT4 codes enter the tensor cores as offset bytes c + 8: the correction
+// 8 sum(digits) per digit column (zero for INT8).
+template <int BITS>
+__device__ __forceinline__ void offset_corr(const int (&dsum)[3], int (&corr)[3]) {
+#pragma unroll
+  for (int d = 0; d < 3; ++d) {
+    int v2 = dsum[d];
+    if (BITS == 4) {
+#pragma unroll
+      for (int off = 16; off; off >>= 1) v2 += __shfl_xor_sync(FULL, v2, off);
+    }
+    corr[d] = BITS == 4 ? 8 * v2 : 0;
+  }
+}
+
+// B fragments (k32 x n8) of one right-hand-side set: column g of lane (g, t)
+// is digit row row_of_g of `dig`.
+template <int D, int BITS>
+__device__ __forceinline__ void load_bfrag(const uint8_t* src, int t, uint32_t (&bfr)[D / 32][2]) {
+  constexpr int NC = D / 32;
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    if (BITS == 4) {
+      const int at = (D / 4) * t + 8 * c;
+      bfr[c][0] = *reinterpret_cast<const uint32_t*>(src + at);
+      bfr[c][1] = *reinterpret_cast<const uint32_t*>(src + at + 4);
+    } else {
+      const int m0 = 2 * c, m1 = 2 * c + 1;
+      const int j0 = m0 < NC ? (D / 8) * t + 4 * m0 : D / 2 + (D / 8) * t + 4 * (m0 - NC);
+      const int j1 = m1 < NC ? (D / 8) * t + 4 * m1 : D / 2 + (D / 8) * t + 4 * (m1 - NC);
+      bfr[c][0] = *reinterpret_cast<const uint32_t*>(src + j0);
+      bfr[c][1] = *reinterpret_cast<const uint32_t*>(src + j1);
+    }
+  }
+}
 
 // One warp's shared-memory stage for one head (byte offsets, all 16-aligned).
 template <int D, bool BF16, int PMAX>
@@ -86,12 +179,14 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
 }
 
 // EXACT: the pool's period equals PMAX (compile-time loop bounds over tokens).
-template <int D, bool BF16, int PMAX, int BITS, bool EXACT>
+// ADAPT: a commit threshold is set: also track the accumulated update's norm
+// and mark the head for an early commit when it reaches the threshold.
+template <int D, bool BF16, int PMAX, int BITS, bool EXACT, bool ADAPT>
 __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, const void* __restrict__ q,
                                             const void* __restrict__ k, const void* __restrict__ v,
                                             const void* __restrict__ alpha,
                                             const void* __restrict__ beta, float* __restrict__ o,
-                                            WarpScratch<D>& scr, const uint8_t* stg, int lane) {
+                                            WarpScratch<D, ADAPT>& scr, const uint8_t* stg, int lane) {
   using ST = Stage<D, BF16, PMAX>;
   constexpr int EPL = D / 32, RB = D / 16, PF = 2;
   constexpr int ESZ = BF16 ? 2 : 4;
@@ -148,11 +243,14 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
       }
     } else if (s == n - 1) {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) part[PMAX + s] = fmaf(qf[e], kf[e], part[PMAX + s]);
+      for (int e = 0; e < EPL; ++e) {
+        part[PMAX + s] = fmaf(qf[e], kf[e], part[PMAX + s]);
+        if (ADAPT) part[s] = fmaf(kf[e], kf[e], part[s]);
+      }
     }
   }
   const float tot = transpose_reduce<2 * PMAX>(part, lane);
-  // lane s < PMAX: gk = k_n . k_s ; lane PMAX + s: q . k_s
+  // lane s < PMAX: gk = k_n . k_s (ADAPT: lane n-1 holds k_n . k_n); lane PMAX + s: q . k_s
 
   // 4. per-token decays / gates, lane s = token s (0-based); lanes >= n neutral
   float al = 1.f, be = 0.f;
@@ -198,31 +296,44 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     }
     acol[tt] = (tt > lane && tt < n) ? bt * run * G : 0.f;
   }
-  if (n == P && lane < PMAX) {         // kept for the period-end factors (step 12)
+  if ((ADAPT || n == P) && lane < PMAX) {   // kept for the period-end factors (step 12)
 #pragma unroll
     for (int tt = 0; tt < PMAX; ++tt) scr.A[tt * PMAX + lane] = acol[tt];
     scr.gsb[0][lane] = gcum;
     scr.gsb[1][lane] = suf;
     scr.gsb[2][lane] = be;
   }
-  // 6. backward substitution (I + A^T) y = w, lane-parallel over s
+  // 6. backward substitution (I + A^T) y = w, lane-parallel over s.
+  //    ADAPT: also the system of the first n-1 tokens for the query k_n with
+  //    w'_s = gamma_{n/s} (k_s . k_n): then zeta = diag(beta) y' gives
+  //    alpha_n S_{n-1} k_n = S~0 a^ + sum_s zeta_s v_s, a^ = gamma_n k_n - b^,
+  //    b^ = sum_s zeta_s gamma_s k_s.
   float acc = w_s;
+  float acc2 = ADAPT && lane < n - 1 ? suf * tot : 0.f;
 #pragma unroll
   for (int tt = PMAX - 1; tt >= 0; --tt) {
     if (tt < n) {
       const float yt = __shfl_sync(FULL, acc, tt);
       if (lane < tt) acc = fmaf(-acol[tt], yt, acc);
     }
+    if (ADAPT && tt < n - 1) {
+      const float yt = __shfl_sync(FULL, acc2, tt);
+      if (lane < tt) acc2 = fmaf(-acol[tt], yt, acc2);
+    }
   }
   const float z = be * acc;              // z_s (0 on lanes >= n)
   const float zk = z * gcum;             // z_s gamma_s
+  const float zeta = be * acc2;          // zeta_s (0 on lanes >= n - 1)
+  const float zetak = zeta * gcum;
 
   // 7. q^ and the buffered-value term, lane-local over its EPL elements
-  float qh[EPL], vt[EPL];
+  float qh[EPL], vt[EPL], bh[EPL], vt2[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
     qh[e] = gamma_n * qf[e];
     vt[e] = 0.f;
+    bh[e] = 0.f;
+    vt2[e] = 0.f;
   }
 #pragma unroll
   for (int s = 0; s < PMAX; ++s) {
@@ -242,90 +353,52 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
         qh[e] = fmaf(-zks, ks[e], qh[e]);
         vt[e] = fmaf(zs, vs[e], vt[e]);
       }
-    }
-  }
-
-  // 8. right-hand side b = q^ (times the column scales) as 22-bit fixed point,
-  //    split into three balanced base-256 digits: b 2^e = d0 + 256 d1 + 65536 d2
-  const bool col = p.axis == PACE_SCALE_COL;
-  float bv[EPL];
-  float m = 0.f;
+      if (ADAPT && s < n - 1) {
+        const float eks = __shfl_sync(FULL, zetak, s);
+        const float es = __shfl_sync(FULL, zeta, s);
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    bv[e] = col ? qh[e] * sc[e] : qh[e];
-    m = fmaxf(m, fabsf(bv[e]));
-  }
-#pragma unroll
-  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
-  int ex = 0;
-  if (m > 0.f && m < INFINITY) ex = max(-120, min(120, 21 - ilogbf(m)));
-  const float up = ldexpf(1.f, ex), down = ldexpf(1.f, -ex);
-  int dsum[3] = {0, 0, 0};
-  uint32_t dw[3] = {0u, 0u, 0u};    // digit bytes of this lane's EPL elements
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    const int Q = __float2int_rn(bv[e] * up);
-    const int d0 = (int)(int8_t)(Q & 0xff);
-    const int r1 = (Q - d0) >> 8;
-    const int d1 = (int)(int8_t)(r1 & 0xff);
-    const int d2 = (r1 - d1) >> 8;
-    dsum[0] += d0; dsum[1] += d1; dsum[2] += d2;
-    dw[0] |= (uint32_t)(d0 & 0xff) << (8 * e);
-    dw[1] |= (uint32_t)(d1 & 0xff) << (8 * e);
-    dw[2] |= (uint32_t)(d2 & 0xff) << (8 * e);
-  }
-  if (BITS == 8) {
-    // natural key-channel order
-#pragma unroll
-    for (int d = 0; d < 3; ++d) {
-      uint8_t* dst = &scr.dig[d][EPL * lane];
-      if (EPL == 4) *reinterpret_cast<uint32_t*>(dst) = dw[d];
-      else if (EPL == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)dw[d];
-      else *dst = (uint8_t)dw[d];
-    }
-  } else {
-    // within each group of 8 key channels: even offsets first, then odd
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const int j = EPL * lane + e, o = j & 7;
-      const int at = (j & ~7) + ((o & 1) ? 4 + (o >> 1) : (o >> 1));
-#pragma unroll
-      for (int d = 0; d < 3; ++d) scr.dig[d][at] = (uint8_t)(dw[d] >> (8 * e));
-    }
-  }
-  // INT4 codes enter the tensor cores as offset bytes c + 8: remove 8 sum(digits)
-  int corr[3] = {0, 0, 0};
-  if (BITS == 4) {
-#pragma unroll
-    for (int d = 0; d < 3; ++d) {
-      int v2 = dsum[d];
-#pragma unroll
-      for (int off = 16; off; off >>= 1) v2 += __shfl_xor_sync(FULL, v2, off);
-      corr[d] = 8 * v2;
-    }
-  }
-  __syncwarp();
-  constexpr int NC = D / 32;           // k32 chunks
-  uint32_t bfr[NC][2];
-  {
-    const uint8_t* src = &scr.dig[g < 3 ? g : 3][0];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      if (BITS == 4) {
-        const int at = (D / 4) * t + 8 * c;
-        bfr[c][0] = *reinterpret_cast<const uint32_t*>(src + at);
-        bfr[c][1] = *reinterpret_cast<const uint32_t*>(src + at + 4);
-      } else {
-        const int m0 = 2 * c, m1 = 2 * c + 1;
-        const int j0 = m0 < NC ? (D / 8) * t + 4 * m0 : D / 2 + (D / 8) * t + 4 * (m0 - NC);
-        const int j1 = m1 < NC ? (D / 8) * t + 4 * m1 : D / 2 + (D / 8) * t + 4 * (m1 - NC);
-        bfr[c][0] = *reinterpret_cast<const uint32_t*>(src + j0);
-        bfr[c][1] = *reinterpret_cast<const uint32_t*>(src + j1);
+        for (int e = 0; e < EPL; ++e) {
+          bh[e] = fmaf(eks, ks[e], bh[e]);
+          vt2[e] = fmaf(es, vs[e], vt2[e]);
+        }
       }
     }
   }
-  const int cA = t == 0 ? corr[0] : corr[2];
-  const int cB = t == 0 ? corr[1] : 0;
+
+  // 8. right-hand sides (times the column scales) as digit rows
+  const bool col = p.axis == PACE_SCALE_COL;
+  float bv[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) bv[e] = col ? qh[e] * sc[e] : qh[e];
+  int dsum[3], corr[3];
+  const float down = rhs_digits<D, EPL, BITS>(bv, &scr.dig[0], lane, dsum);
+  offset_corr<BITS>(dsum, corr);
+  float down_a = 0.f, down_b = 0.f;
+  int corr_a[3] = {0, 0, 0}, corr_b[3] = {0, 0, 0};
+  if constexpr (ADAPT) {
+    float av[EPL], bw[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const float ah = gamma_n * kf[e] - bh[e];
+      av[e] = col ? ah * sc[e] : ah;
+      bw[e] = col ? bh[e] * sc[e] : bh[e];
+    }
+    down_a = rhs_digits<D, EPL, BITS>(av, &scr.dig[4], lane, dsum);
+    offset_corr<BITS>(dsum, corr_a);
+    down_b = rhs_digits<D, EPL, BITS>(bw, &scr.dig[8], lane, dsum);
+    offset_corr<BITS>(dsum, corr_b);
+  }
+  __syncwarp();
+  constexpr int NC = D / 32;           // k32 chunks
+  // columns 0..2: q^ digits; ADAPT: 4..6 a^ digits (second product: 0..2 b^)
+  uint32_t bfr[NC][2], bfr2[NC][2];
+  load_bfrag<D, BITS>(&scr.dig[g < 3 || (ADAPT && g >= 4 && g < 7) ? g : 3][0], t, bfr);
+  if constexpr (ADAPT) load_bfrag<D, BITS>(&scr.dig[g < 3 ? 8 + g : 3][0], t, bfr2);
+  // accumulator columns 2t, 2t+1 of lane t: (d0, d1) for even t, (d2, -) for odd t
+  const int cA = t == 0 ? corr[0] : t == 1 ? corr[2] : t == 2 ? corr_a[0] : corr_a[2];
+  const int cB = t == 0 ? corr[1] : t == 2 ? corr_a[1] : 0;
+  const int cA2 = t == 0 ? corr_b[0] : t == 1 ? corr_b[2] : 0;
+  const int cB2 = t == 0 ? corr_b[1] : 0;
 
   // 9. y = S~0 (codes) x b on the int8 tensor cores (exact int32), 16 rows at a time
   // (unrolled by the prefetch depth only: a smaller loop body keeps the
@@ -337,7 +410,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     const int r = r0 + rr;
     RowBlock<D, BITS> cur = rbuf[rr];
     if (r + PF < RB) rbuf[rr].load(rec, r + PF, g, t);
-    int d[4] = {0, 0, 0, 0};
+    int d[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
       uint32_t a[4];
@@ -348,16 +421,19 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
         a[2] = ((w0 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
         a[3] = ((w1 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
         mma_u8s8(d, a, bfr[c][0], bfr[c][1]);
+        if constexpr (ADAPT) mma_u8s8(d2, a, bfr2[c][0], bfr2[c][1]);
       } else {
         a[0] = cur.w[0][2 * c];
         a[1] = cur.w[1][2 * c];
         a[2] = cur.w[0][2 * c + 1];
         a[3] = cur.w[1][2 * c + 1];
         mma_s8s8(d, a, bfr[c][0], bfr[c][1]);
+        if constexpr (ADAPT) mma_s8s8(d2, a, bfr2[c][0], bfr2[c][1]);
       }
     }
-    // columns 0, 1, 2 = digits: lane t = 0 holds d0, d1; lane t = 1 holds d2
-    const float wB = t == 0 ? 256.f : 0.f, wA = t == 0 ? 1.f : 65536.f;
+    // digit columns: lane t = 0 holds d0, d1 and lane t = 1 holds d2 of q^
+    // (ADAPT: lanes 2, 3 the same of a^; second product: lanes 0, 1 of b^)
+    const float wB = (t & 1) == 0 ? 256.f : 0.f, wA = (t & 1) == 0 ? 1.f : 65536.f;
     float pg = wA * (float)(d[0] - cA) + wB * (float)(d[1] - cB);
     float ph = wA * (float)(d[2] - cA) + wB * (float)(d[3] - cB);
     pg += __shfl_down_sync(FULL, pg, 1);
@@ -365,6 +441,20 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     if (t == 0) {
       scr.y[16 * r + g] = pg * down;
       scr.y[16 * r + g + 8] = ph * down;
+    }
+    if constexpr (ADAPT) {
+      if (t == 2) {
+        scr.ya[16 * r + g] = pg * down_a;
+        scr.ya[16 * r + g + 8] = ph * down_a;
+      }
+      float pg2 = wA * (float)(d2[0] - cA2) + wB * (float)(d2[1] - cB2);
+      float ph2 = wA * (float)(d2[2] - cA2) + wB * (float)(d2[3] - cB2);
+      pg2 += __shfl_down_sync(FULL, pg2, 1);
+      ph2 += __shfl_down_sync(FULL, ph2, 1);
+      if (t == 0) {
+        scr.yb[16 * r + g] = pg2 * down_b;
+        scr.yb[16 * r + g + 8] = ph2 * down_b;
+      }
     }
   }
   __syncwarp();
@@ -383,6 +473,33 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     else op[0] = out[0];
   }
 
+  // 10a. ADAPT: the accumulated update Delta_n = S_n - gamma_n S~0 by
+  //      |Delta_n|^2 = alpha_n^2 |Delta_{n-1}|^2 + 2 u_n . e^ + |u_n|^2 |k_n|^2,
+  //      u_n = beta_n (v_n - alpha_n S_{n-1} k_n), e^ = alpha_n Delta_{n-1} k_n
+  //      = sum_s zeta_s v_s - S~0 b^; the head is due when it reaches tau^2
+  bool commit_now = n == P;
+  float norm2 = 0.f;
+  if constexpr (ADAPT) {
+    float ue = 0.f, uu = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const float sa = col ? scr.ya[EPL * lane + e] : scr.ya[EPL * lane + e] * sc[e];
+      const float sb = col ? scr.yb[EPL * lane + e] : scr.yb[EPL * lane + e] * sc[e];
+      const float u = b_n * (vf[e] - (sa + vt2[e]));
+      ue = fmaf(u, vt2[e] - sb, ue);
+      uu = fmaf(u, u, uu);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      ue += __shfl_xor_sync(FULL, ue, off);
+      uu += __shfl_xor_sync(FULL, uu, off);
+    }
+    const float kk = __shfl_sync(FULL, tot, n - 1);
+    const float prev = n > 1 ? reinterpret_cast<const float*>(stg + ST::G)[P * P + P] : 0.f;
+    norm2 = fmaxf(a_n * a_n * prev + 2.f * ue + uu * kk, 0.f);
+    commit_now = commit_now || norm2 >= p.tau2;
+  }
+
   // 11. buffer the token: k, v, alpha, beta, its Gram row; then fill = n
   uint8_t* row = const_cast<uint8_t*>(kv_head) + (size_t)(n - 1) * row_elems * ESZ;
   k_raw.store(row, (size_t)EPL * lane);
@@ -395,13 +512,15 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     ra.store(abp, 0);
     rb2.store(abp, 1);
   }
-  if (n < P && lane < n - 1) const_cast<float*>(gram_head)[(n - 1) * P + lane] = tot;
+  if (!commit_now && lane < n - 1) const_cast<float*>(gram_head)[(n - 1) * P + lane] = tot;
+  if (ADAPT && !commit_now && lane == 0) const_cast<float*>(gram_head)[P * P + P] = norm2;
 
-  // 12. period end (n == P): replace the Gram block by the commit's chunk-form
-  //     factors W[t][s] = gamma_{P/t} T[t][s] beta_s, T = (I + A)^{-1} (lane s
-  //     solves column s by forward substitution), followed by gamma_s, the
-  //     largest |k| of the period and the largest stored scale
-  if (n == P) {
+  // 12. period end (n == P, or marked early): replace the Gram block by the
+  //     commit's chunk-form factors W[t][s] = gamma_{n/t} T[t][s] beta_s,
+  //     T = (I + A)^{-1} (lane s solves column s by forward substitution;
+  //     zero beyond n), followed by gamma_s (gamma_n beyond n), the largest
+  //     |k| of the period and the largest stored scale
+  if (commit_now) {
     float km = 0.f, sm = 0.f;
     {
       float x[EPL];
@@ -448,7 +567,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     }
   }
   __syncwarp();
-  if (lane == 0) p.fill[head] = n;
+  if (lane == 0) p.fill[head] = commit_now && n < P ? (n | PACE_FILL_COMMIT) : n;
 }
 
 // Bulk-copy head `head`'s staged inputs into `stg` (lane 0 only): q, k, v, the
@@ -478,7 +597,7 @@ __device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill
   }
 }
 
-template <int D, bool BF16, int PMAX, bool EXACT>
+template <int D, bool BF16, int PMAX, bool EXACT, bool ADAPT>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_step_kernel(PoolDev p, const void* __restrict__ q, const void* __restrict__ k,
                        const void* __restrict__ v, const void* __restrict__ alpha,
@@ -488,10 +607,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   uint8_t* stages = smem_raw + (size_t)wib * NS * ST::BYTES;
-  WarpScratch<D>& scr =
-      reinterpret_cast<WarpScratch<D>*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES)[wib];
+  WarpScratch<D, ADAPT>& scr =
+      reinterpret_cast<WarpScratch<D, ADAPT>*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES)[wib];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES +
-                                              kWarpsPerBlock * sizeof(WarpScratch<D>)) + NS * wib;
+                                              kWarpsPerBlock * sizeof(WarpScratch<D, ADAPT>)) + NS * wib;
   for (int i = lane; i < D; i += 32) scr.dig[3][i] = 0;
   const int n_heads = sp.nb * p.H;   // work items of this launch
   const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
@@ -550,9 +669,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int n = nprev + 1;
     if (p.bits[head % p.H] == 4)
-      decode_head<D, BF16, PMAX, 4, EXACT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
+      decode_head<D, BF16, PMAX, 4, EXACT, ADAPT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
     else
-      decode_head<D, BF16, PMAX, 8, EXACT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
+      decode_head<D, BF16, PMAX, 8, EXACT, ADAPT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
   }
 }
 
@@ -569,13 +688,13 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, bool BF16, int PMAX, bool EXACT>
+template <int D, bool BF16, int PMAX, bool EXACT, bool ADAPT = false>
 cudaError_t launch_t(const PoolDev& p, const Span& sp, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
   using ST = Stage<D, BF16, PMAX>;
-  const size_t smem = (size_t)kWarpsPerBlock * (ST::N * ST::BYTES + sizeof(WarpScratch<D>) +
+  const size_t smem = (size_t)kWarpsPerBlock * (ST::N * ST::BYTES + sizeof(WarpScratch<D, ADAPT>) +
                                                 ST::N * sizeof(uint64_t));
-  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX, EXACT>,
+  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX, EXACT, ADAPT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long heads = (long)sp.nb * p.H;
@@ -583,14 +702,19 @@ cudaError_t launch_t(const PoolDev& p, const Span& sp, const void* q, const void
   long blocks = (heads + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const long cap = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 2) * sm_count();
   if (blocks > cap) blocks = cap;
-  decode_step_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, kThreads, smem, st>>>(p, q, k, v, alpha,
-                                                                                     beta, o, sp);
+  decode_step_kernel<D, BF16, PMAX, EXACT, ADAPT><<<(unsigned)blocks, kThreads, smem, st>>>(
+      p, q, k, v, alpha, beta, o, sp);
   return cudaGetLastError();
 }
 
 template <int D, bool BF16>
 cudaError_t launch_p(const PoolDev& p, const Span& sp, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
+  if (p.adaptive) {   // commit threshold set: the period is the buffer's capacity
+    if (p.P <= 4) return launch_t<D, BF16, 4, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+    if (p.P <= 8) return launch_t<D, BF16, 8, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+    return launch_t<D, BF16, 16, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+  }
   switch (p.P) {
     case 4: return launch_t<D, BF16, 4, true>(p, sp, q, k, v, alpha, beta, o, st);
     case 8: return launch_t<D, BF16, 8, true>(p, sp, q, k, v, alpha, beta, o, st);

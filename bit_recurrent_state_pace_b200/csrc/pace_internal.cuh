@@ -32,7 +32,15 @@ struct PoolDev {
   uint8_t bits[PACE_MAX_HEADS];       // 4 or 8
   uint8_t order[PACE_MAX_HEADS];      // head indices, the 4-bit heads first
   int32_t H4;                         // number of 4-bit heads
+  float tau2;                         // commit threshold squared (+inf: fixed period)
+  int32_t adaptive;                   // tau2 finite
 };
+
+// A head's buffer is due for a commit: full, or marked by the decode step
+// (which marks only heads holding at least one token).
+__host__ __device__ inline bool commit_due(int32_t fill, int32_t P) {
+  return fill == P || ((fill & PACE_FILL_COMMIT) != 0 && (fill & 0xff) > 0);
+}
 
 // The slots a launch works on, and how many blocks per SM it may occupy
 // (fewer than the default leaves room for a launch on another stream).

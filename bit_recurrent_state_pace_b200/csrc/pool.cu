@@ -2,6 +2,8 @@
 #include <new>
 #include <string.h>
 
+#include <cmath>
+
 #include "pace_internal.cuh"
 
 struct pace_pool {
@@ -158,6 +160,8 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
     for (int h = 0; h < desc->num_heads; ++h)
       if (desc->head_bits[h] != 4) dv.order[n4++] = (uint8_t)h;
   }
+  dv.tau2 = INFINITY;
+  dv.adaptive = 0;
   for (int h = 0; h < desc->num_heads; ++h) {
     dv.rec_off[h] = (uint32_t)L.rec_off[h];
     dv.bits[h] = desc->head_bits[h];
@@ -222,6 +226,13 @@ pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, cons
                              const void* alpha, const void* beta, float* o, void* stream) {
   if (!pool) return PACE_ERR_INVALID_ARG;
   return pace_decode_step_range(pool, 0, pool->dev.B, 0, q, k, v, alpha, beta, o, stream);
+}
+
+pace_status pace_set_commit_threshold(pace_pool* pool, float tau) {
+  if (!pool || !(tau >= 0.f)) return PACE_ERR_INVALID_ARG;   // NaN fails the comparison
+  pool->dev.adaptive = std::isfinite(tau) ? 1 : 0;
+  pool->dev.tau2 = pool->dev.adaptive ? tau * tau : INFINITY;
+  return PACE_OK;
 }
 
 pace_status pace_commit_period_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,

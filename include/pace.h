@@ -53,6 +53,11 @@ typedef enum {
                                           that head's output row is NaN, nothing stored */
 #define PACE_FLAG_TIMEOUT        0x8u  /* a bounded wait inside a kernel gave up */
 
+/* Fill-counter bit: the head's accumulated update reached the pool's commit
+ * threshold (pace_set_commit_threshold) before its buffer filled; the low
+ * bits still count its buffered tokens. */
+#define PACE_FILL_COMMIT 0x100
+
 /* Scale axis ([P2] "Channel-Aligned Encoding"; [P4] TL;DR (2)).
  * COL: one scale per key channel j, shared by the d_v entries S[:, j].
  * ROW: one scale per value channel i, shared by the d_k entries S[i, :]. */
@@ -98,8 +103,12 @@ typedef struct {
  *          T[s][s'] beta_s' with T = (I + A)^{-1}, then the P decay products
  *          gamma_s, then max |k_s[j]| over the period's keys and the largest
  *          stored scale of the head.  q is not stored: no later step reads
- *          an old query.
- * aux    : fill counters int32 [B][H] (tokens in each head's buffer), then at
+ *          an old query.  With a commit threshold set, float P*P + P of the
+ *          block holds, while the period fills, the squared norm of the
+ *          accumulated update, and the factors above are written for the n
+ *          buffered tokens by the step that marks the head (zero beyond n).
+ * aux    : fill counters int32 [B][H] (tokens in each head's buffer, plus
+ *          PACE_FILL_COMMIT when the head is due early), then at
  *          byte offset round_up(4*B*H, 256) the uint32 status word.
  * All three regions must be 256-byte aligned.
  */
@@ -151,9 +160,30 @@ pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, cons
                              const void* alpha, const void* beta, float* o, void* stream);
 
 /*
+ * Adaptive period ([P4] "Research angle": round when the accumulated update
+ * norm crosses a threshold rather than every k tokens).  With tau set, the
+ * decode step also tracks, for each head, the Frobenius norm of the update
+ * accumulated since the last rounding,
+ *   Delta_n = S_n - gamma_n S~0 = sum_s gamma_{n/s} u_s k_s^T
+ * (the writes; the decay alone needs no re-encoding), by the recursion
+ *   |Delta_n|^2 = alpha_n^2 |Delta_{n-1}|^2 + 2 alpha_n u_n . (Delta_{n-1} k_n)
+ *                 + |u_n|^2 |k_n|^2,   u_n = beta_n (v_n - alpha_n S_{n-1} k_n),
+ * whose vectors come from the same pass over the stored codes as o_n
+ * (fp32; decisions within rounding of the threshold may go either way).
+ * When |Delta_n| >= tau and n < P the step marks the head (fill = n |
+ * PACE_FILL_COMMIT); pace_commit_period then commits it with its n tokens,
+ * and a decode step on a marked head is skipped like one on a full buffer.
+ * tau = +inf (the default) is the fixed period P; tau = 0 commits after
+ * every token.  A negative or NaN tau is PACE_ERR_INVALID_ARG.  Host-only:
+ * applies to launches enqueued after the call.
+ */
+pace_status pace_set_commit_threshold(pace_pool* pool, float tau);
+
+/*
  * Period end ([P4] flowchart "every k tokens -> State update, chunked, high
  * precision -> 4-bit encode, per-column scales"; 8-bit heads from TL;DR (3)).
- * For every head whose buffer holds P tokens: dequantise the stored state,
+ * For every head whose buffer holds P tokens (or is marked PACE_FILL_COMMIT
+ * with n tokens): dequantise the stored state,
  * apply the P buffered tokens in one chunked (UT/WY) update in fp32, encode
  * the result with fresh absmax scales at the head's bit width, write it back
  * in place, and empty the buffer.  Heads with fewer than P tokens are left
