@@ -43,6 +43,9 @@ def parse_args():
     ap.add_argument("--axis", choices=["col", "row"], default=None, help="override the scale axis")
     ap.add_argument("--prefill-tokens", type=int, default=64,
                     help="tokens of the chunked fp32 prefill measured after the decode (0: skip)")
+    ap.add_argument("--commit-threshold", default=None,
+                    help="also measure the adaptive period with this threshold on the accumulated "
+                         "update's Frobenius norm ('auto': the median after 3 tokens)")
     ap.add_argument("--bits-from-gates", action="store_true",
                     help="choose the 8-bit heads from the prefill gates (slowest mean decay) "
                          "instead of the workload's seeded choice")
@@ -459,6 +462,12 @@ def run_pace(args, rank: int, world: int):
     if not args.no_e2e:
         e2e = run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag)
 
+    # ---- adaptive period: every token is a decode step and a commit launch for
+    #      the heads marked by it; the pool is restored afterwards
+    adaptive = None
+    if args.commit_threshold is not None and stag is None:
+        adaptive = run_adaptive(args, pace, pool, w, toks, outs, stream, world, dev, mk)
+
     # ---- chunked fp32 prefill of T tokens into the whole pool (after the decode
     #      numbers: it rewrites the pool); not part of the headline step
     prefill = None
@@ -520,9 +529,94 @@ def run_pace(args, rank: int, world: int):
             "device_status": status,
             "comparison": compare,
             "prefill": prefill,
+            "adaptive": adaptive,
             "cpu_baseline": cpu_base,
         }
         print(json.dumps(line), flush=True)
+
+
+def gram_norm2(pool, w):
+    """The accumulated-update norms^2 the tracking decode keeps in each head's
+    factor block (float P*P + P of block [b][h] of the buffer's G region)."""
+    import torch
+    ru = lambda x, a: (x + a - 1) // a * a
+    esz = 2 if w.io_dtype == "bf16" else 4
+    BH, P = w.B * w.H, w.P
+    ab_off = ru(BH * P * (w.d_k + w.d_v) * esz, 256)
+    g_off = ru(ab_off + BH * ru(2 * P * esz, 16), 256)
+    g_stride = ru(4 * (P * (P + 1) + 2), 16)
+    g = pool.buffer[g_off:g_off + BH * g_stride].view(BH, g_stride).view(torch.float32)
+    return g[:, P * P + P]
+
+
+def run_adaptive(args, pace, pool, w, toks, outs, stream, world, dev, mk):
+    import torch
+    from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+    P, BH = w.P, w.B * w.H
+    sp = stream.cuda_stream
+    saved = pool.state.clone()
+    torch.cuda.synchronize()
+    assert int(pool.fill().count_nonzero()) == 0
+
+    def restore():
+        pool.state.copy_(saved)
+        pool.fill().zero_()
+        torch.cuda.synchronize()
+
+    if args.commit_threshold == "auto":
+        pool.set_commit_threshold(1e30)   # track, never mark
+        for n in range(3):
+            x = toks[n]
+            pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n], sp)
+        tau = float(torch.sqrt(torch.median(gram_norm2(pool, w))))
+        rule = "median accumulated-update norm after 3 tokens"
+        restore()
+    else:
+        tau, rule = float(args.commit_threshold), "given"
+    pool.set_commit_threshold(tau)
+
+    def token(n, ev=None):
+        x = toks[n % P]
+        if ev is not None:
+            ev[0].record(stream)
+        pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n % P], sp)
+        if ev is not None:
+            ev[1].record(stream)
+        pace.pace_commit_period(pool.handle, sp)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for n in range(args.warmup * P):
+        token(n)
+    torch.cuda.synchronize()
+    ntok = args.steps * P
+    evs = [(mk(), mk(), mk()) for _ in range(ntok)]
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = mk(), mk()
+    a.record(stream)
+    for n in range(ntok):
+        token(n, evs[n])
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    dec_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    com_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # commits per head-token, counted outside the timed region
+    commits = 0
+    for n in range(2 * P):
+        x = toks[n % P]
+        pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n % P], sp)
+        f = pool.fill()
+        commits += int(((f & pace.PACE_FILL_COMMIT) != 0).sum() + (f == P).sum())
+        pace.pace_commit_period(pool.handle, sp)
+    status = pool.status()
+    pool.set_commit_threshold(float("inf"))
+    restore()
+    return {"tau": tau, "tau_rule": rule, "value": aggregate_rate(BH * ntok, world, ms),
+            "unit": "head-tokens/s", "ms_per_token": ms / ntok, "decode_ms": dec_ms,
+            "commit_ms_per_launch": com_ms, "mean_tokens_per_commit": BH * 2 * P / max(commits, 1),
+            "gpu_launches": 2 * ntok, "status": status}
 
 
 def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag=None):
