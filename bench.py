@@ -77,13 +77,26 @@ def measured_peaks():
         return HBM_FALLBACK_GBS, "fallback"
 
 
-def kernel_source_digest():
+KERNEL_SOURCES = {"decode_step": "decode_kernels.cu", "commit": "commit_kernels.cu"}
+
+
+def kernel_source_digest(kernel: str) -> str:
+    """sha256 (16 hex digits) of a kernel's source file and every csrc header
+    it includes, directly or not: what a DRAM-traffic record depends on."""
+    import re
     csrc = os.path.join(ROOT, "bit_recurrent_state_pace_b200", "csrc")
+    todo, seen = [KERNEL_SOURCES[kernel]], []
+    while todo:
+        fn = todo.pop()
+        if fn in seen or not os.path.exists(os.path.join(csrc, fn)):
+            continue
+        seen.append(fn)
+        with open(os.path.join(csrc, fn)) as f:
+            todo += re.findall(r'^#include "([^"/]+)"', f.read(), flags=re.M)
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    for fn in sorted(seen):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -393,12 +406,10 @@ def run_pace(args, rank: int, world: int):
     hbm, peak_kind = measured_peaks()
     dec_gbs = dec_avg_bytes / (dec_avg_ms * 1e-3) / 1e9
     com_gbs = com_bytes / (com_avg_ms * 1e-3) / 1e9
-    digest = kernel_source_digest()
+    digest = {kern: kernel_source_digest(kern) for kern in KERNEL_SOURCES}
     dominant = "decode_step" if dec_avg_ms * P >= com_avg_ms else "commit"
-    if dominant == "decode_step":
-        ach, traffic = dec_gbs, ncu_traffic("decode_step", digest)
-    else:
-        ach, traffic = com_gbs, ncu_traffic("commit", digest)
+    ach = dec_gbs if dominant == "decode_step" else com_gbs
+    traffic = ncu_traffic(dominant, digest[dominant])
 
     from bit_recurrent_state_pace_b200.ranks import aggregate_rate
     lockstep_value = aggregate_rate(BH * P * args.steps, world, elapsed_ms)

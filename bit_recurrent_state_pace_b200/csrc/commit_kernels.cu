@@ -656,8 +656,8 @@ cudaError_t launch_p(const PoolDev& p, const Span& sp, cudaStream_t st) {
     case 8: return launch_t<D, BF16, 8, true>(p, sp, st);
     case 16: return launch_t<D, BF16, 16, true>(p, sp, st);
   }
-  if (p.P < 4) return launch_t<D, BF16, 4, false>(p, sp, st);
-  if (p.P < 8) return launch_t<D, BF16, 8, false>(p, sp, st);
+  if (p.P <= 4) return launch_t<D, BF16, 4, false>(p, sp, st);
+  if (p.P <= 8) return launch_t<D, BF16, 8, false>(p, sp, st);
   return launch_t<D, BF16, 16, false>(p, sp, st);
 }
 
