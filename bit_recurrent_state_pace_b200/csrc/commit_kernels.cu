@@ -87,11 +87,15 @@ struct alignas(16) Smem {
   int slow[2];                                    // by head parity: exact-encode fallback needed
 };
 
-// First head index >= from (stepping by step, below end) due for a commit.
-__device__ __forceinline__ int find_full(const PoolDev& p, int from, int step, int end) {
-  int hd = from;
-  while (hd < end && !commit_due(p.fill[hd], p.P)) hd += step;
-  return hd;
+// First head index >= from (stepping by step, below end) due for a commit,
+// or end.  The 32 lanes of the calling warp test 32 candidates at a time.
+__device__ __forceinline__ int find_full_warp(const PoolDev& p, int from, int step, int end, int lane) {
+  for (int base = from; base < end; base += 32 * step) {
+    const int hd = base + lane * step;
+    const unsigned m = __ballot_sync(FULL, hd < end && commit_due(p.fill[hd], p.P));
+    if (m) return base + (__ffs((int)m) - 1) * step;
+  }
+  return end;
 }
 
 template <int D, bool BF16, int PMAX>
@@ -557,22 +561,30 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
   // heads [b0 H, (b0 + nb) H) of this launch; n_heads is the end index
   const int first_head = sp.b0 * p.H;
   const int n_heads = (sp.b0 + sp.nb) * p.H;
-  // thread ISS (idle during the scale pass) issues every bulk copy; it keeps
-  // the candidate head two ahead and its fill count
+  // thread ISS (idle during the scale pass) issues every bulk copy.  Its
+  // warp finds the first due heads 32 at a time (a launch may have none);
+  // afterwards ISS keeps the candidate after the staged heads and its fill
+  // count, loaded one head ahead, so a due candidate costs no wait.
   constexpr int ISS = C::THREADS / 2;
+  const bool iss_warp = (tid >> 5) == (ISS >> 5);
+  const int lane = tid & 31;
   int cand = n_heads, cand_fill = 0;
-  if (tid == ISS) {
-    for (int i = 0; i < 3; ++i) mbar_init(&sm.bar[i], 1);
-    fence_mbar_init();
-    int h = find_full(p, first_head + blockIdx.x, gridDim.x, n_heads);
-    for (int i = 0; i < 3; ++i) sm.hq[i] = n_heads;
+  if (iss_warp) {
+    if (tid == ISS) {
+      for (int i = 0; i < 3; ++i) mbar_init(&sm.bar[i], 1);
+      fence_mbar_init();
+      for (int i = 0; i < 3; ++i) sm.hq[i] = n_heads;
+    }
+    int h = find_full_warp(p, first_head + blockIdx.x, gridDim.x, n_heads, lane);
     for (int i = 0; i < 2; ++i) {
-      sm.hq[i] = h;
-      if (h < n_heads) {
-        sm.hn[i] = p.fill[h] & 0xff;
-        issue_head<D, BF16, PMAX>(p, h, sm, i);
-        h = find_full(p, h + gridDim.x, gridDim.x, n_heads);
+      if (tid == ISS) {
+        sm.hq[i] = h;
+        if (h < n_heads) {
+          sm.hn[i] = p.fill[h] & 0xff;
+          issue_head<D, BF16, PMAX>(p, h, sm, i);
+        }
       }
+      if (h < n_heads) h = find_full_warp(p, h + gridDim.x, gridDim.x, n_heads, lane);
     }
     cand = h;
     if (cand < n_heads) cand_fill = p.fill[cand];
@@ -587,14 +599,16 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     const bool ok = mbar_wait_bounded(&sm.bar[s], (parity >> s) & 1u, p.flags);
     parity ^= 1u << s;
     const int s2 = s == 0 ? 2 : s - 1;   // slot of the head two ahead (held the previous head)
-    auto issue_next = [&]() {
+    auto issue_next = [&]() {   // every thread of the block calls it
       if (tid == ISS) {
-        int nxt = cand;
-        if (nxt < n_heads && !commit_due(cand_fill, p.P))
-          nxt = find_full(p, nxt + gridDim.x, gridDim.x, n_heads);
+        int nxt = cand, nfill = cand_fill;
+        while (nxt < n_heads && !commit_due(nfill, p.P)) {
+          nxt += gridDim.x;
+          nfill = nxt < n_heads ? p.fill[nxt] : 0;
+        }
         sm.hq[s2] = nxt;
         if (nxt < n_heads) {
-          sm.hn[s2] = (nxt == cand ? cand_fill : p.fill[nxt]) & 0xff;
+          sm.hn[s2] = nfill & 0xff;
           issue_head<D, BF16, PMAX>(p, nxt, sm, s2);
         }
         cand = nxt < n_heads ? nxt + gridDim.x : n_heads;
