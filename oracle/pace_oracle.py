@@ -52,6 +52,13 @@ Pages cited (by title and section):
    rounded after token n when ``||Delta_n||_F >= tau`` and in any case when
    its buffer of P tokens is full.  ``update_norm2`` writes the definition
    out; ``pace_run_adaptive`` is the per-head driver.
+7. Pure-write window.  [P3], section "PW：让近期写入走“纯净通道”": the
+   most recent writes are kept apart from the low-bit history as FP8 vector
+   pairs (k, v) that take full part in the state transition, and a pair is
+   merged into the low-bit history only when it leaves the window of S
+   steps.  ``e4m3`` is the FP8 format (E4M3: 4 exponent bits, bias 7, 3
+   mantissa bits, largest finite 448), rounding to nearest with ties to even
+   and saturating at +-448; ``pw_run`` is the windowed driver.
 
 Everything here is fp64 except the quantiser, which takes the fp32 state and
 reproduces the fp32/fp16 operations of the encoding one by one with numpy's
@@ -477,3 +484,58 @@ def pace_run_adaptive(state: PoolState, tokens: Sequence[Dict[str, np.ndarray]],
         norms.append(norm2)
     final = PoolState(codes, scales, state.bits, state.axis)
     return outs, final, rounded, norms, flags
+
+
+# --------------------------------------------------------------------------
+# Pure-write window, [P3] section "PW：让近期写入走“纯净通道”": the last S
+# writes stay outside the low-bit history as FP8 (k, v) pairs that take full
+# part in the state transition; the oldest pair is merged into the history
+# (which is then rounded) when it leaves the window.
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3(x) -> np.ndarray:
+    """Round to FP8 E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits,
+    no infinities; subnormal quantum 2^-9): the nearest representable value,
+    ties to the even mantissa, saturating at +-448; NaN stays NaN; the sign of
+    zero is kept.  Returned as fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, E = np.frexp(a)                      # a = m 2^E, m in [0.5, 1)
+    e = np.maximum(E - 1, -6)               # binade exponent, normals from 2^-6
+    q = np.ldexp(1.0, e - 3)                # quantum: 3 mantissa bits
+    with np.errstate(invalid="ignore"):
+        r = np.round(a / q) * q             # a / q is exact; round() ties to even
+    r = np.minimum(r, E4M3_MAX)
+    r = np.where(np.isnan(x), np.nan, r)
+    return np.copysign(r, x)
+
+
+def pw_run(state: PoolState, tokens: Sequence[Dict[str, np.ndarray]], S: int, step=gdn_step):
+    """Decode ``tokens`` with a pure-write window of S steps, every head in step.
+
+    Each token's k and v are rounded to E4M3 and join the window; the output
+    is S_t q_t with S_t the dequantised history advanced exactly (fp64)
+    through every pair of the window.  When the window then holds S pairs,
+    its oldest pair is applied to the history alone, the history is rounded
+    (fp32, then each head's bit width) and the pair leaves the window.
+
+    Returns (outputs per token [N, d_v], final history PoolState, the tokens
+    still in the window, flags).
+    """
+    window: List[Dict[str, np.ndarray]] = []
+    outs, flags = [], 0
+    for tok in tokens:
+        window.append(dict(tok, k=e4m3(tok["k"]), v=e4m3(tok["v"])))
+        S_t = state.dequantized()
+        for w in window:
+            S_t, o = step(S_t, tok["q"], w["k"], w["v"], w["alpha"], w["beta"])
+        outs.append(o)
+        if len(window) == S:
+            old = window.pop(0)
+            S_h, _ = step(state.dequantized(), tok["q"], old["k"], old["v"], old["alpha"], old["beta"])
+            state, f = commit(S_h, state.bits, state.axis)
+            flags |= f
+    return outs, state, window, flags

@@ -551,3 +551,110 @@ def check_adaptive_driver_per_head(pace_run_adaptive, chunk_form, PoolState, qua
     # the threshold, not the buffer, must end most periods here
     full = sum(bool(r[i]) for r in rounded for i in range(N))
     assert n_rounded == full and full > N * T // P
+
+
+# ---------------- pure-write window ----------------
+
+def e4m3_code_values():
+    """Every E4M3 bit pattern decoded from its fields: sign, 4 exponent bits
+    (bias 7), 3 mantissa bits; exponent 0 is subnormal (m 2^-9); S.1111.111 is
+    NaN.  Returns the finite values, one per code."""
+    vals = []
+    for c in range(256):
+        s, E, m = c >> 7, (c >> 3) & 15, c & 7
+        if E == 15 and m == 7:
+            continue
+        v = m * 2.0 ** -9 if E == 0 else (1 + m / 8) * 2.0 ** (E - 7)
+        vals.append(-v if s else v)
+    return np.array(vals)
+
+
+def check_e4m3(e4m3, seed=0):
+    vals = e4m3_code_values()
+    assert vals.max() == 448.0 and np.min(np.abs(vals[vals != 0])) == 2.0 ** -9
+    # representable values are fixed points
+    assert np.array_equal(e4m3(vals), vals)
+    # brute force: the nearest finite value, ties to the even mantissa, over
+    # random values and every midpoint between neighbours
+    pos = np.unique(np.abs(vals))
+    codes = {float(v): i for i, v in enumerate(pos)}    # mantissa parity follows the index
+    rng = np.random.default_rng(seed)
+    xs = np.concatenate([rng.standard_normal(2000) * 4.0, rng.uniform(-460, 460, 500),
+                         rng.standard_normal(500) * 0.01, (pos[1:] + pos[:-1]) / 2,
+                         -(pos[1:] + pos[:-1]) / 2])
+    for x in xs:
+        a = abs(x)
+        if a >= 448.0:
+            want = 448.0
+        else:
+            d = np.abs(pos - a)
+            best = np.nonzero(d == d.min())[0]
+            want = pos[best[0]] if len(best) == 1 else pos[[b for b in best if codes[float(pos[b])] % 2 == 0][0]]
+        got = e4m3(np.array([x]))[0]
+        assert got == np.copysign(want, x), (x, got, want)
+    # saturation, signed zero, NaN
+    assert e4m3(np.array([1e6, -500.0]))[0] == 448.0 and e4m3(np.array([-500.0]))[0] == -448.0
+    assert np.signbit(e4m3(np.array([-0.0]))[0]) and np.isnan(e4m3(np.array([np.nan]))[0])
+
+
+def check_pw_limits(pw_run, per_token_rounding, sequential, e4m3, PoolState, quantize, seed=0):
+    """A window of one step is per-token rounding of the E4M3-rounded writes;
+    a window longer than the stream never merges, so it is the exact
+    recurrence from the stored state over those writes."""
+    rng = np.random.default_rng(seed)
+    N, d_v, d_k = 5, 8, 8
+    bits = [4, 8, 4, 8, 4]
+    for axis in ("col", "row"):
+        codes, scales = _random_pool_state(rng, N, d_v, d_k, bits, axis, quantize)
+        st = PoolState(codes, scales, bits, axis)
+        toks = random_tokens(rng, N, 9, d_k, d_v)
+        for tk in toks:
+            tk["v"] = tk["v"] * 3.0
+        rounded = [dict(tk, k=e4m3(tk["k"]), v=e4m3(tk["v"])) for tk in toks]
+        o_w, fin_w, window, _ = pw_run(st, toks, 1)
+        o_p, fin_p = per_token_rounding(st, rounded)
+        assert not window
+        for x, y in zip(o_w, o_p):
+            assert np.array_equal(x, y)
+        assert all(np.array_equal(a, b) for a, b in zip(fin_w.codes, fin_p.codes))
+        o_w, fin_w, window, _ = pw_run(st, toks, len(toks) + 1)
+        _, o_s = sequential(st.dequantized(), rounded)
+        assert len(window) == len(toks)
+        for x, y in zip(o_w, o_s):
+            assert np.allclose(x, y, rtol=1e-12, atol=1e-12)
+        assert all(np.array_equal(a, b) for a, b in zip(fin_w.codes, st.codes))
+
+
+def check_pw_replay(pw_run, chunk_form, e4m3, PoolState, quantize, dequantize, seed=0):
+    """A window of S = 3 replayed in chunk form: the output of every token is
+    the chunk-form readout of the history through the window's pairs, and
+    the history after a merge is the encoding of one step of its oldest pair."""
+    rng = np.random.default_rng(seed)
+    N, d_v, d_k, S, T = 4, 8, 8, 3, 10
+    bits = [4, 8, 4, 4]
+    axis = "col"
+    codes, scales = _random_pool_state(rng, N, d_v, d_k, bits, axis, quantize)
+    st = PoolState(codes, scales, bits, axis)
+    toks = random_tokens(rng, N, T, d_k, d_v)
+    o_w, fin, window, _ = pw_run(st, toks, S)
+    H = st.dequantized()
+    hc, hs = list(codes), list(scales)
+    win = []
+    for t, tk in enumerate(toks):
+        win.append(dict(tk, k=e4m3(tk["k"]), v=e4m3(tk["v"])))
+        K = np.stack([w["k"] for w in win], 1)
+        V = np.stack([w["v"] for w in win], 1)
+        A = np.stack([w["alpha"] for w in win], 1)
+        B = np.stack([w["beta"] for w in win], 1)
+        _, _, o = chunk_form(H, K, V, A, B, tk["q"])
+        assert np.allclose(o_w[t], o, rtol=1e-10, atol=1e-12), t
+        if len(win) == S:
+            old = win.pop(0)
+            Sh, _, _ = chunk_form(H, old["k"][:, None], old["v"][:, None], old["alpha"][:, None],
+                                  old["beta"][:, None])
+            for i in range(N):
+                c, s, _ = quantize(Sh[i:i + 1].astype(np.float32), bits[i], axis)
+                hc[i], hs[i] = c[0], s[0]
+            H = np.stack([dequantize(c, s, axis) for c, s in zip(hc, hs)]).astype(np.float64)
+    assert len(window) == S - 1
+    assert all(np.array_equal(a, b) for a, b in zip(fin.codes, hc))

@@ -249,3 +249,66 @@ def test_adaptive_driver_mutant_is_caught(kind):
               or _fails(ck.check_adaptive_driver_per_head, run, orc.chunk_form, orc.PoolState,
                         orc.quantize, orc.dequantize))
     assert caught == (kind != "none"), kind
+
+
+# ---------------- pure-write window mutants ----------------
+
+def _e4m3_factory(kind):
+    def e4m3(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        _, E = np.frexp(a)
+        e = np.maximum(E - 1, -7 if kind == "subnormal_quantum" else -6)
+        q = np.ldexp(1.0, e - (2 if kind == "two_mantissa_bits" else 3))
+        with np.errstate(invalid="ignore"):
+            r = (np.floor(a / q + 0.5) if kind == "ties_away" else np.round(a / q)) * q
+        if kind != "no_saturation":
+            r = np.minimum(r, 448.0)
+        r = np.where(np.isnan(x), np.nan, r)
+        return np.copysign(r, x)
+    return e4m3
+
+
+E4M3_MUTANTS = ["subnormal_quantum", "two_mantissa_bits", "ties_away", "no_saturation"]
+
+
+@pytest.mark.parametrize("kind", E4M3_MUTANTS + ["none"])
+def test_e4m3_mutant_is_caught(kind):
+    assert _fails(ck.check_e4m3, _e4m3_factory(kind)) == (kind != "none"), kind
+
+
+def _pw_factory(kind):
+    def run(state, tokens, S, step=orc.gdn_step):
+        window, outs = [], []
+        for tok in tokens:
+            k = tok["k"] if kind == "k_not_rounded" else orc.e4m3(tok["k"])
+            window.append(dict(tok, k=k, v=orc.e4m3(tok["v"])))
+            if kind == "merge_before_readout" and len(window) == S:
+                old = window.pop(0)
+                S_h, _ = step(state.dequantized(), tok["q"], old["k"], old["v"], old["alpha"], old["beta"])
+                state, _ = orc.commit(S_h, state.bits, state.axis)
+            S_t = state.dequantized()
+            o = np.einsum("nij,nj->ni", S_t, np.asarray(tok["q"], dtype=np.float64))
+            for w in window:
+                S_t, o = step(S_t, tok["q"], w["k"], w["v"], w["alpha"], w["beta"])
+            outs.append(o)
+            limit = S + 1 if kind == "window_one_longer" else S
+            if kind != "merge_before_readout" and len(window) == limit:
+                old = window.pop(-1 if kind == "merge_newest" else 0)
+                S_h, _ = step(state.dequantized(), tok["q"], old["k"], old["v"], old["alpha"], old["beta"])
+                state, _ = orc.commit(S_h, state.bits, state.axis)
+        return outs, state, window, 0
+    return run
+
+
+PW_MUTANTS = ["k_not_rounded", "merge_before_readout", "window_one_longer", "merge_newest"]
+
+
+@pytest.mark.parametrize("kind", PW_MUTANTS + ["none"])
+def test_pw_mutant_is_caught(kind):
+    run = _pw_factory(kind)
+    caught = (_fails(ck.check_pw_limits, run, orc.per_token_rounding, orc.sequential, orc.e4m3,
+                     orc.PoolState, orc.quantize)
+              or _fails(ck.check_pw_replay, run, orc.chunk_form, orc.e4m3, orc.PoolState, orc.quantize,
+                        orc.dequantize))
+    assert caught == (kind != "none"), kind

@@ -145,3 +145,17 @@ def test_adaptive_period_limits():
 def test_adaptive_period_replayed_per_head_in_chunk_form():
     ck.check_adaptive_driver_per_head(orc.pace_run_adaptive, orc.chunk_form, orc.PoolState,
                                       orc.quantize, orc.dequantize)
+
+
+def test_e4m3_against_its_code_table():
+    ck.check_e4m3(orc.e4m3)
+
+
+def test_pure_write_window_limits():
+    ck.check_pw_limits(orc.pw_run, orc.per_token_rounding, orc.sequential, orc.e4m3, orc.PoolState,
+                       orc.quantize)
+
+
+def test_pure_write_window_replayed_in_chunk_form():
+    ck.check_pw_replay(orc.pw_run, orc.chunk_form, orc.e4m3, orc.PoolState, orc.quantize,
+                       orc.dequantize)
