@@ -26,7 +26,7 @@ __all__ = [
     "pace_pool_load", "pace_pool_export", "pace_decode_step", "pace_commit_period",
     "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
     "pace_select_head_bits", "pace_prefill", "pace_prefill_range", "pace_host_staging_bytes",
-    "pace_decode_host", "pace_set_commit_threshold",
+    "pace_decode_host", "pace_set_commit_threshold", "pace_window_scratch_bytes", "pace_window_step",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -80,6 +80,8 @@ def _load():
         "pace_prefill": [P, I64, P, P, P, P, P, F32p, P],
         "pace_host_staging_bytes": [P, Sp],
         "pace_set_commit_threshold": [P, ctypes.c_float],
+        "pace_window_scratch_bytes": [P, Sp],
+        "pace_window_step": [P, P, P, P, P, P, F32p, P, P],
         "pace_decode_host": [P, I32, P, P, P, P, P, P, P, P, P, P],
         "pace_prefill_range": [P, I32, I32, I64, P, P, P, P, P, F32p, P],
         "pace_select_head_bits": [P, I32, I32, P],
@@ -185,6 +187,17 @@ def pace_decode_step(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
 
 def pace_commit_period(handle: int, stream=None) -> None:
     _check("pace_commit_period", lib.pace_commit_period(handle, _stream(stream)))
+
+
+def pace_window_scratch_bytes(handle: int) -> int:
+    n = ctypes.c_size_t()
+    _check("pace_window_scratch_bytes", lib.pace_window_scratch_bytes(handle, ctypes.byref(n)))
+    return n.value
+
+
+def pace_window_step(handle: int, q, k, v, alpha, beta, o, scratch, stream=None) -> None:
+    _check("pace_window_step", lib.pace_window_step(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                                    _ptr(beta), _ptr(o), _ptr(scratch), _stream(stream)))
 
 
 def pace_set_commit_threshold(handle: int, tau: float) -> None:
@@ -371,6 +384,16 @@ class PacePool:
     def prefill(self, q, k, v, alpha, beta, o=None, stream=None) -> Optional[torch.Tensor]:
         """T tokens [T][B][H][d] through the chunked fp32 prefill; returns o."""
         pace_prefill(self.handle, int(q.shape[0]), q, k, v, alpha, beta, o, stream)
+        return o
+
+    def window_step(self, q, k, v, alpha, beta, o=None, stream=None) -> torch.Tensor:
+        """One pure-write-window step (window length = P) for every head."""
+        if getattr(self, "_wscratch", None) is None:
+            self._wscratch = torch.empty(pace_window_scratch_bytes(self.handle), dtype=torch.uint8,
+                                         device=self.state.device)
+        if o is None:
+            o = torch.empty(self.B, self.H, self.d_v, dtype=torch.float32, device=self.state.device)
+        pace_window_step(self.handle, q, k, v, alpha, beta, o, self._wscratch, stream)
         return o
 
     def set_commit_threshold(self, tau: float) -> None:

@@ -5,6 +5,7 @@
 #include <cmath>
 
 #include "pace_internal.cuh"
+#include "window.cuh"
 
 struct pace_pool {
   pace::PoolDev dev;
@@ -349,6 +350,36 @@ pace_status pace_decode_host(pace_pool* pool, int32_t n_tokens, const void* h_q,
     if (landed[j]) cudaEventDestroy(landed[j]);
     if (computed[j]) cudaEventDestroy(computed[j]);
   }
+  return from_cuda(e);
+}
+
+pace_status pace_window_scratch_bytes(const pace_pool* pool, size_t* bytes) {
+  if (!pool || !bytes) return PACE_ERR_INVALID_ARG;
+  const size_t BH = (size_t)pool->dev.B * pool->dev.H, esz = pool->dev.io == PACE_IO_BF16 ? 2 : 4;
+  *bytes = round_up(BH * pool->dev.d_k * esz, 256) + round_up(BH * pool->dev.d_v * esz, 256);
+  return PACE_OK;
+}
+
+pace_status pace_window_step(pace_pool* pool, const void* q, const void* k, const void* v,
+                             const void* alpha, const void* beta, float* o, void* d_scratch,
+                             void* stream) {
+  if (!pool || !q || !k || !v || !alpha || !beta || !o || !d_scratch) return PACE_ERR_INVALID_ARG;
+  if (!aligned(d_scratch, 256) || pool->dev.adaptive) return PACE_ERR_INVALID_ARG;
+  const size_t BH = (size_t)pool->dev.B * pool->dev.H, esz = pool->dev.io == PACE_IO_BF16 ? 2 : 4;
+  uint8_t* k8 = static_cast<uint8_t*>(d_scratch);
+  uint8_t* v8 = k8 + round_up(BH * pool->dev.d_k * esz, 256);
+  cudaStream_t st = as_stream(stream);
+  const pace::Span all{0, pool->dev.B, 0};
+  cudaError_t e = pace::launch_e4m3_round(k, k8, (int64_t)(BH * pool->dev.d_k), pool->dev.io, st);
+  if (e == cudaSuccess) e = pace::launch_e4m3_round(v, v8, (int64_t)(BH * pool->dev.d_v), pool->dev.io, st);
+  if (e == cudaSuccess) e = pace::launch_decode_step(pool->dev, all, q, k8, v8, alpha, beta, o, st);
+  if (e == cudaSuccess) e = pace::launch_window_prepare(pool->dev, st);
+  if (e == cudaSuccess) {
+    pace::PoolDev one = pool->dev;   // commits the marked heads with their own token count
+    one.adaptive = 1;
+    e = pace::launch_commit(one, all, st);
+  }
+  if (e == cudaSuccess) e = pace::launch_window_shift(pool->dev, st);
   return from_cuda(e);
 }
 

@@ -286,6 +286,27 @@ pace_status pace_decode_host(pace_pool* pool, int32_t n_tokens, const void* h_q,
                              void* d_staging, void* stream, void* h2d_stream, void* d2h_stream);
 
 /*
+ * Pure-write window ("低比特量化新突破：GGA+PW让线性注意力长文本生成更准更短",
+ * section "PW：让近期写入走“纯净通道”": the most recent writes stay apart from
+ * the low-bit history as FP8 (k, v) pairs that take full part in the state
+ * transition, and a pair is merged into the history when it leaves the
+ * window).  The pool's buffer is the window and P its length S.  One step
+ * for every head: k and v are rounded to FP8 E4M3 (nearest, ties to even,
+ * saturating at +-448; kept in the io dtype, which holds every E4M3 value
+ * exactly), o_t = S_t q_t is read out from the stored history and the
+ * window as pace_decode_step does, and a head whose window then holds P
+ * pairs applies its oldest pair alone to the history, re-encodes it, and
+ * drops that pair (fill returns to P - 1).  Inputs and o as
+ * pace_decode_step; d_scratch: device memory of pace_window_scratch_bytes
+ * bytes, 256-byte aligned, for the rounded k and v.  A pool with a commit
+ * threshold set is PACE_ERR_INVALID_ARG.  Enqueues only.
+ */
+pace_status pace_window_scratch_bytes(const pace_pool* pool, size_t* bytes);
+pace_status pace_window_step(pace_pool* pool, const void* q, const void* k, const void* v,
+                             const void* alpha, const void* beta, float* o, void* d_scratch,
+                             void* stream);
+
+/*
  * Chunked fp32 prefill (the chunked prefill kernels that [P2] "Periodic
  * Rounding" cites; [P4] flowchart "State update, chunked, high precision").
  * For every head of the slots (all of them, or [slot_begin, slot_begin +
