@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--commit-threshold", default=None,
                     help="also measure the adaptive period with this threshold on the accumulated "
                          "update's Frobenius norm ('auto': the median after 3 tokens)")
+    ap.add_argument("--window", action="store_true",
+                    help="also measure the pure-write window (pace_window_step, window = P)")
     ap.add_argument("--bits-from-gates", action="store_true",
                     help="choose the 8-bit heads from the prefill gates (slowest mean decay) "
                          "instead of the workload's seeded choice")
@@ -479,6 +481,12 @@ def run_pace(args, rank: int, world: int):
     if args.commit_threshold is not None and stag is None:
         adaptive = run_adaptive(args, pace, pool, w, toks, outs, stream, world, dev, mk)
 
+    # ---- pure-write window: every token is a window step (the oldest pair of
+    #      a full window is merged into the history); the pool is restored
+    window = None
+    if args.window and stag is None:
+        window = run_window(args, pace, pool, w, toks, outs, stream, world, dev, mk)
+
     # ---- chunked fp32 prefill of T tokens into the whole pool (after the decode
     #      numbers: it rewrites the pool); not part of the headline step
     prefill = None
@@ -541,6 +549,7 @@ def run_pace(args, rank: int, world: int):
             "comparison": compare,
             "prefill": prefill,
             "adaptive": adaptive,
+            "window": window,
             "cpu_baseline": cpu_base,
         }
         print(json.dumps(line), flush=True)
@@ -628,6 +637,41 @@ def run_adaptive(args, pace, pool, w, toks, outs, stream, world, dev, mk):
             "unit": "head-tokens/s", "ms_per_token": ms / ntok, "decode_ms": dec_ms,
             "commit_ms_per_launch": com_ms, "mean_tokens_per_commit": BH * 2 * P / max(commits, 1),
             "gpu_launches": 2 * ntok, "status": status}
+
+
+def run_window(args, pace, pool, w, toks, outs, stream, world, dev, mk):
+    import torch
+    from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+    P, BH = w.P, w.B * w.H
+    saved = pool.state.clone()
+    torch.cuda.synchronize()
+    assert int(pool.fill().count_nonzero()) == 0
+
+    def token(n):
+        x = toks[n % P]
+        pool.window_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n % P], stream)
+
+    for n in range(max(args.warmup, 1) * P):   # the window is full from here on
+        token(n)
+    torch.cuda.synchronize()
+    ntok = args.steps * P
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = mk(), mk()
+    a.record(stream)
+    for n in range(ntok):
+        token(n)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    status = pool.status()
+    pool.state.copy_(saved)
+    pool.fill().zero_()
+    torch.cuda.synchronize()
+    return {"window": P, "value": aggregate_rate(BH * ntok, world, ms), "unit": "head-tokens/s",
+            "ms_per_token": ms / ntok, "gpu_launches": 6 * ntok, "status": status,
+            "note": "every token: E4M3 rounding of k and v, the decode step, and the merge of each "
+                    "head's oldest pair (one-token commit of every head, then the window shift)"}
 
 
 def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag=None):
