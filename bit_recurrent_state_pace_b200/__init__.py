@@ -54,7 +54,7 @@ class _Desc(ctypes.Structure):
     _fields_ = [("num_slots", ctypes.c_int32), ("num_heads", ctypes.c_int32),
                 ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("period", ctypes.c_int32),
                 ("scale_axis", ctypes.c_int32), ("io_dtype", ctypes.c_int32),
-                ("head_bits", ctypes.POINTER(ctypes.c_uint8))]
+                ("head_bits", ctypes.POINTER(ctypes.c_uint8)), ("buffer_e4m3", ctypes.c_int32)]
 
 
 def _load():
@@ -136,25 +136,27 @@ def _stream(stream) -> Optional[int]:
     return int(stream)
 
 
-def _desc(B, H, d_k, d_v, P, axis, io, head_bits) -> Tuple[_Desc, ctypes.Array]:
+def _desc(B, H, d_k, d_v, P, axis, io, head_bits, buffer_e4m3=0) -> Tuple[_Desc, ctypes.Array]:
     vals = [int(b) for b in head_bits]
     bits_arr = (ctypes.c_uint8 * max(len(vals), 1))(*vals)
-    d = _Desc(B, H, d_k, d_v, P, axis, io, ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_uint8)))
+    d = _Desc(B, H, d_k, d_v, P, axis, io, ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_uint8)),
+              int(buffer_e4m3))
     return d, bits_arr
 
 
 # ---------------------------------------------------------------- C names
 
-def pace_pool_bytes(B, H, d_k, d_v, P, axis, io, head_bits) -> Tuple[int, int, int]:
-    d, keep = _desc(B, H, d_k, d_v, P, axis, io, head_bits)
+def pace_pool_bytes(B, H, d_k, d_v, P, axis, io, head_bits, buffer_e4m3=0) -> Tuple[int, int, int]:
+    d, keep = _desc(B, H, d_k, d_v, P, axis, io, head_bits, buffer_e4m3)
     a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     _check("pace_pool_bytes", lib.pace_pool_bytes(ctypes.byref(d), ctypes.byref(a), ctypes.byref(b),
                                                    ctypes.byref(c)))
     return a.value, b.value, c.value
 
 
-def pace_init_pool(B, H, d_k, d_v, P, axis, io, head_bits, state, buffer, aux, stream=None) -> int:
-    d, keep = _desc(B, H, d_k, d_v, P, axis, io, head_bits)
+def pace_init_pool(B, H, d_k, d_v, P, axis, io, head_bits, state, buffer, aux, stream=None,
+                   buffer_e4m3=0) -> int:
+    d, keep = _desc(B, H, d_k, d_v, P, axis, io, head_bits, buffer_e4m3)
     out = ctypes.c_void_p()
     _check("pace_init_pool", lib.pace_init_pool(ctypes.byref(d), _ptr(state), _ptr(buffer), _ptr(aux),
                                                  _stream(stream), ctypes.byref(out)))
@@ -322,18 +324,21 @@ class PacePool:
     """
 
     def __init__(self, B: int, H: int, d_k: int, d_v: int, P: int, head_bits: Sequence[int],
-                 axis: str = "col", io: str = "bf16", device="cuda", stream=None):
+                 axis: str = "col", io: str = "bf16", device="cuda", stream=None,
+                 buffer_e4m3: bool = False):
         self.B, self.H, self.d_k, self.d_v, self.P = B, H, d_k, d_v, P
+        self.buffer_e4m3 = bool(buffer_e4m3)
         self.head_bits = [int(b) for b in head_bits]
         self.axis = PACE_SCALE_COL if axis == "col" else PACE_SCALE_ROW
         self.io = PACE_IO_BF16 if io == "bf16" else PACE_IO_F32
         self.io_torch = torch.bfloat16 if io == "bf16" else torch.float32
-        sb, bb, ab = pace_pool_bytes(B, H, d_k, d_v, P, self.axis, self.io, self.head_bits)
+        sb, bb, ab = pace_pool_bytes(B, H, d_k, d_v, P, self.axis, self.io, self.head_bits,
+                                     int(self.buffer_e4m3))
         self.state = torch.empty(sb, dtype=torch.uint8, device=device)
         self.buffer = torch.zeros(bb, dtype=torch.uint8, device=device)
         self.aux = torch.empty(ab, dtype=torch.uint8, device=device)
         self.handle = pace_init_pool(B, H, d_k, d_v, P, self.axis, self.io, self.head_bits,
-                                     self.state, self.buffer, self.aux, stream)
+                                     self.state, self.buffer, self.aux, stream, int(self.buffer_e4m3))
         self.slot_stride = pace_pool_layout(self.handle, 0)[2]
 
     def __del__(self):

@@ -33,6 +33,7 @@
 // f16 magic-number conversion (1032 + c, 1152 + c) and packed in place.
 #include <type_traits>
 
+#include "e4m3.cuh"
 #include "tma.cuh"
 #include "update_common.cuh"
 
@@ -98,14 +99,15 @@ __device__ __forceinline__ int find_full_warp(const PoolDev& p, int from, int st
   return end;
 }
 
-template <int D, bool BF16, int PMAX>
+template <int D, bool BF16, int PMAX, bool R8>
 __device__ __forceinline__ void issue_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, int s) {
   using C = Cfg<D, BF16, PMAX>;
   const int h = head % p.H, b = head / p.H;
   const uint32_t rec_bytes = (uint32_t)record_bytes(D, D, p.bits[h], D);
-  const uint32_t kv_bytes = (uint32_t)(p.P * 2 * D * C::ESZ);
+  constexpr uint32_t row = 2 * D * (R8 ? 1 : C::ESZ);   // bytes of a buffered row
+  const uint32_t kv_bytes = (uint32_t)p.P * row;
   const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
-  const uint8_t* kv = p.kv + (size_t)head * p.P * 2 * D * C::ESZ;
+  const uint8_t* kv = p.kv + (size_t)head * p.P * row;
   const uint8_t* ab = p.ab + (size_t)head * p.ab_stride;
   const uint8_t* gr = p.gram + (size_t)head * p.gram_stride;
   uint8_t* dst = sm.slot[s];
@@ -113,7 +115,7 @@ __device__ __forceinline__ void issue_head(const PoolDev& p, int head, Smem<D, B
   mbar_arrive_expect_tx(&sm.bar[s], rec_bytes + kv_bytes + p.ab_stride + p.gram_stride);
   tma_load_1d(dst, rec, rec_bytes, &sm.bar[s]);
   for (int r = 0; r < p.P; ++r)
-    tma_load_1d(dst + C::REC + r * C::ROWS, kv + (size_t)r * 2 * D * C::ESZ, 2 * D * C::ESZ, &sm.bar[s]);
+    tma_load_1d(dst + C::REC + r * C::ROWS, kv + (size_t)r * row, row, &sm.bar[s]);
   tma_load_1d(dst + C::REC + C::KVB, ab, p.ab_stride, &sm.bar[s]);
   tma_load_1d(dst + C::REC + C::KVB + C::ABB, gr, p.gram_stride, &sm.bar[s]);
 }
@@ -151,7 +153,8 @@ __device__ __forceinline__ void load_rows_smem(RowBlock<D, BITS>& rb, const uint
 // Returns false (every thread) when the staged copies of this head did not
 // arrive in time (ok == false in some thread); nothing is written then.
 // n_tok: the head's buffered tokens (P, or fewer for a head marked early).
-template <int D, bool BF16, int PMAX, int BITS, bool EXACT, class Issue>
+// R8: the buffered rows are E4M3 bytes.
+template <int D, bool BF16, int PMAX, int BITS, bool EXACT, bool R8, class Issue>
 __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm, const uint8_t* slot,
                             int n_tok, bool ok, int parity_bit, Issue&& issue_next) {
   using C = Cfg<D, BF16, PMAX>;
@@ -200,7 +203,7 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
 #pragma unroll
         for (int pos = 0; pos < 4; ++pos) {
           const int j = jof<D, BITS>(tt, ks, pos);
-          const float kv = io_at(s_kv + s * C::ROWS, j, BF16);
+          const float kv = row_at<R8>(s_kv + s * C::ROWS, j, BF16);
           const float xv = (col ? kv * __half2float(__ushort_as_half(s_sc[j])) : kv) * upx;
           hv[pos] = __float2half_rn(xv);
           lv[pos] = __float2half_rn(xv - __half2float(hv[pos]));
@@ -233,7 +236,7 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
           const int seg = sigma / PMAX, s2 = sigma % PMAX;
           __half h = __ushort_as_half((unsigned short)0);
           if (seg < C::NSEG && s2 < P) {
-            const float kv = io_at(s_kv + s2 * C::ROWS, j, BF16);
+            const float kv = row_at<R8>(s_kv + s2 * C::ROWS, j, BF16);
             h = __float2half_rn(kv);
             if (seg == 2) h = __float2half_rn(kv - __half2float(h));
           }
@@ -280,8 +283,8 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       ro[x][0] = ro[x][1] = 0.f;
       if (s < P) {
         const float gs = gam[s];
-        ro[x][0] = io_at(s_kv + s * C::ROWS, D + i0, BF16) - gs * ((xacc[x][0] + xacc[x][1]) * s0);
-        ro[x][1] = io_at(s_kv + s * C::ROWS, D + i1, BF16) - gs * ((xacc[x][2] + xacc[x][3]) * s1);
+        ro[x][0] = row_at<R8>(s_kv + s * C::ROWS, D + i0, BF16) - gs * ((xacc[x][0] + xacc[x][1]) * s0);
+        ro[x][1] = row_at<R8>(s_kv + s * C::ROWS, D + i1, BF16) - gs * ((xacc[x][2] + xacc[x][3]) * s1);
       }
     }
 #pragma unroll
@@ -551,7 +554,7 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
   return true;
 }
 
-template <int D, bool BF16, int PMAX, bool EXACT>
+template <int D, bool BF16, int PMAX, bool EXACT, bool R8>
 __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     commit_kernel(PoolDev p, Span sp) {
   using C = Cfg<D, BF16, PMAX>;
@@ -581,7 +584,7 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
         sm.hq[i] = h;
         if (h < n_heads) {
           sm.hn[i] = p.fill[h] & 0xff;
-          issue_head<D, BF16, PMAX>(p, h, sm, i);
+          issue_head<D, BF16, PMAX, R8>(p, h, sm, i);
         }
       }
       if (h < n_heads) h = find_full_warp(p, h + gridDim.x, gridDim.x, n_heads, lane);
@@ -609,7 +612,7 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
         sm.hq[s2] = nxt;
         if (nxt < n_heads) {
           sm.hn[s2] = nfill & 0xff;
-          issue_head<D, BF16, PMAX>(p, nxt, sm, s2);
+          issue_head<D, BF16, PMAX, R8>(p, nxt, sm, s2);
         }
         cand = nxt < n_heads ? nxt + gridDim.x : n_heads;
         if (cand < n_heads) cand_fill = p.fill[cand];
@@ -617,9 +620,9 @@ __global__ void __launch_bounds__(Cfg<D, BF16, PMAX>::THREADS, 2)
     };
     const bool done =
         p.bits[head % p.H] == 4
-            ? commit_head<D, BF16, PMAX, 4, EXACT>(p, head, sm, sm.slot[s], sm.hn[s], ok, iter & 1,
+            ? commit_head<D, BF16, PMAX, 4, EXACT, R8>(p, head, sm, sm.slot[s], sm.hn[s], ok, iter & 1,
                                                    issue_next)
-            : commit_head<D, BF16, PMAX, 8, EXACT>(p, head, sm, sm.slot[s], sm.hn[s], ok, iter & 1,
+            : commit_head<D, BF16, PMAX, 8, EXACT, R8>(p, head, sm, sm.slot[s], sm.hn[s], ok, iter & 1,
                                                    issue_next);
     if (!done) {   // a bounded wait gave up: let the copies in flight land, then leave
       if (tid == ISS)
@@ -646,11 +649,11 @@ int sm_count_dev() {
   return cached[dev];
 }
 
-template <int D, bool BF16, int PMAX, bool EXACT>
+template <int D, bool BF16, int PMAX, bool EXACT, bool R8 = false>
 cudaError_t launch_t(const PoolDev& p, const Span& sp, cudaStream_t st) {
   using C = Cfg<D, BF16, PMAX>;
   const size_t smem = sizeof(Smem<D, BF16, PMAX>);
-  cudaError_t e = cudaFuncSetAttribute(commit_kernel<D, BF16, PMAX, EXACT>,
+  cudaError_t e = cudaFuncSetAttribute(commit_kernel<D, BF16, PMAX, EXACT, R8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long heads = (long)sp.nb * p.H;
@@ -658,12 +661,22 @@ cudaError_t launch_t(const PoolDev& p, const Span& sp, cudaStream_t st) {
   long blocks = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 2) * sm_count_dev() *
                 (D == 128 ? 1 : D == 64 ? 2 : 4);
   if (blocks > heads) blocks = heads;
-  commit_kernel<D, BF16, PMAX, EXACT><<<(unsigned)blocks, C::THREADS, smem, st>>>(p, sp);
+  commit_kernel<D, BF16, PMAX, EXACT, R8><<<(unsigned)blocks, C::THREADS, smem, st>>>(p, sp);
   return cudaGetLastError();
 }
 
 template <int D, bool BF16>
 cudaError_t launch_p(const PoolDev& p, const Span& sp, cudaStream_t st) {
+  if (p.row8) {   // E4M3 buffered rows
+    if (!p.adaptive) switch (p.P) {
+      case 4: return launch_t<D, BF16, 4, true, true>(p, sp, st);
+      case 8: return launch_t<D, BF16, 8, true, true>(p, sp, st);
+      case 16: return launch_t<D, BF16, 16, true, true>(p, sp, st);
+    }
+    if (p.P <= 4) return launch_t<D, BF16, 4, false, true>(p, sp, st);
+    if (p.P <= 8) return launch_t<D, BF16, 8, false, true>(p, sp, st);
+    return launch_t<D, BF16, 16, false, true>(p, sp, st);
+  }
   // heads marked early hold fewer than P tokens: per-head token counts
   if (!p.adaptive) switch (p.P) {
     case 4: return launch_t<D, BF16, 4, true>(p, sp, st);

@@ -32,6 +32,7 @@
 //  * The small n x n chunk algebra runs lane-parallel over tokens with warp
 //    shuffles; k.k dot products of earlier buffered tokens are cached in the
 //    buffer's Gram block, so each step computes only the 2n-1 new ones.
+#include "e4m3.cuh"
 #include "frag.cuh"
 #include "tma.cuh"
 
@@ -158,6 +159,21 @@ struct Stage {
   static constexpr int N = 2 * 8 * 2 * BYTES <= 160 * 1024 ? 2 : 1;
 };
 
+// EPL consecutive elements (from element index elem) of buffered rows: io
+// dtype, or E4M3 bytes (R8).
+template <int EPL, bool BF16, bool R8>
+__device__ __forceinline__ void load_row(const uint8_t* base, size_t elem, float (&out)[EPL]) {
+  if constexpr (R8) {
+    const uint8_t* p = base + elem;
+    const uint32_t w = EPL == 4 ? *reinterpret_cast<const uint32_t*>(p)
+                     : EPL == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(p) : (uint32_t)*p;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) out[e] = e4m3_value(w >> (8 * e));
+  } else {
+    load_f<EPL, BF16>(base, elem, out);
+  }
+}
+
 // Lane L ends with the warp-wide sum of value index (L mod V).
 template <int V>
 __device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
@@ -181,7 +197,9 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[V], int lane) {
 // EXACT: the pool's period equals PMAX (compile-time loop bounds over tokens).
 // ADAPT: a commit threshold is set: also track the accumulated update's norm
 // and mark the head for an early commit when it reaches the threshold.
-template <int D, bool BF16, int PMAX, int BITS, bool EXACT, bool ADAPT>
+// R8: buffered k, v are E4M3 bytes; the token's k, v are rounded to E4M3 as
+// they are buffered and used.
+template <int D, bool BF16, int PMAX, int BITS, bool EXACT, bool ADAPT, bool R8>
 __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, const void* __restrict__ q,
                                             const void* __restrict__ k, const void* __restrict__ v,
                                             const void* __restrict__ alpha,
@@ -209,8 +227,8 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   load_f<EPL, BF16>(stg + ST::Q, e0, qf);
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
-    kf[e] = k_raw.get(e);
-    vf[e] = v_raw.get(e);
+    kf[e] = R8 ? e4m3_round(k_raw.get(e)) : k_raw.get(e);
+    vf[e] = R8 ? e4m3_round(v_raw.get(e)) : v_raw.get(e);
   }
   const float a_n = load_io(alpha, head, BF16 ? PACE_IO_BF16 : PACE_IO_F32);
   const float b_n = load_io(beta, head, BF16 ? PACE_IO_BF16 : PACE_IO_F32);
@@ -226,7 +244,8 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
 
   // 3. dot products with the buffered keys: k_n.k_s and q.k_s
   const size_t row_elems = 2 * (size_t)D;
-  const uint8_t* kv_head = p.kv + (size_t)head * P * row_elems * ESZ;
+  constexpr int RESZ = R8 ? 1 : ESZ;   // bytes per buffered element
+  const uint8_t* kv_head = p.kv + (size_t)head * P * row_elems * RESZ;
   const uint8_t* kv_stg = stg + ST::KV;
   float part[2 * PMAX];
 #pragma unroll
@@ -235,7 +254,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   for (int s = 0; s < PMAX; ++s) {
     if (s < n - 1) {
       float ks[EPL];
-      load_f<EPL, BF16>(kv_stg, s * row_elems + (size_t)EPL * lane, ks);
+      load_row<EPL, BF16, R8>(kv_stg, s * row_elems + (size_t)EPL * lane, ks);
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
         part[s] = fmaf(kf[e], ks[e], part[s]);
@@ -342,8 +361,8 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
       const float zs = __shfl_sync(FULL, z, s);
       float ks[EPL], vs[EPL];
       if (s < n - 1) {
-        load_f<EPL, BF16>(kv_stg, s * row_elems + (size_t)EPL * lane, ks);
-        load_f<EPL, BF16>(kv_stg, s * row_elems + D + (size_t)EPL * lane, vs);
+        load_row<EPL, BF16, R8>(kv_stg, s * row_elems + (size_t)EPL * lane, ks);
+        load_row<EPL, BF16, R8>(kv_stg, s * row_elems + D + (size_t)EPL * lane, vs);
       } else {
 #pragma unroll
         for (int e = 0; e < EPL; ++e) { ks[e] = kf[e]; vs[e] = vf[e]; }
@@ -501,9 +520,30 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   }
 
   // 11. buffer the token: k, v, alpha, beta, its Gram row; then fill = n
-  uint8_t* row = const_cast<uint8_t*>(kv_head) + (size_t)(n - 1) * row_elems * ESZ;
-  k_raw.store(row, (size_t)EPL * lane);
-  v_raw.store(row, D + (size_t)EPL * lane);
+  uint8_t* row = const_cast<uint8_t*>(kv_head) + (size_t)(n - 1) * row_elems * RESZ;
+  if constexpr (R8) {
+    uint32_t wk = 0u, wv = 0u;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      wk |= (uint32_t)e4m3_code(k_raw.get(e)) << (8 * e);
+      wv |= (uint32_t)e4m3_code(v_raw.get(e)) << (8 * e);
+    }
+    uint8_t* pk = row + (size_t)EPL * lane;
+    uint8_t* pv = row + D + (size_t)EPL * lane;
+    if (EPL == 4) {
+      *reinterpret_cast<uint32_t*>(pk) = wk;
+      *reinterpret_cast<uint32_t*>(pv) = wv;
+    } else if (EPL == 2) {
+      *reinterpret_cast<uint16_t*>(pk) = (uint16_t)wk;
+      *reinterpret_cast<uint16_t*>(pv) = (uint16_t)wv;
+    } else {
+      *pk = (uint8_t)wk;
+      *pv = (uint8_t)wv;
+    }
+  } else {
+    k_raw.store(row, (size_t)EPL * lane);
+    v_raw.store(row, D + (size_t)EPL * lane);
+  }
   if (lane == 0) {
     Raw<1, BF16> ra, rb2;
     ra.load(alpha, head);
@@ -527,8 +567,18 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
 #pragma unroll
       for (int s = 0; s < PMAX; ++s) {
         if (s < n) {
-          load_f<EPL, BF16>(s < n - 1 ? stg + ST::KV : stg + ST::K,
-                            s < n - 1 ? s * row_elems + (size_t)EPL * lane : (size_t)EPL * lane, x);
+          if constexpr (R8) {
+            if (s < n - 1) {
+              load_row<EPL, BF16, true>(stg + ST::KV, s * row_elems + (size_t)EPL * lane, x);
+            } else {   // the token's own k, again from the stage, rounded as buffered
+              load_f<EPL, BF16>(stg + ST::K, (size_t)EPL * lane, x);
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) x[e] = e4m3_round(x[e]);
+            }
+          } else {
+            load_f<EPL, BF16>(s < n - 1 ? stg + ST::KV : stg + ST::K,
+                              s < n - 1 ? s * row_elems + (size_t)EPL * lane : (size_t)EPL * lane, x);
+          }
 #pragma unroll
           for (int e = 0; e < EPL; ++e) km = fmaxf(km, fabsf(x[e]));
         }
@@ -573,7 +623,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
 // Bulk-copy head `head`'s staged inputs into `stg` (lane 0 only): q, k, v, the
 // scales, and -- when `fill` tokens (0 < fill < P) are buffered -- its rows,
 // gates and Gram block.  Completes on `bar` with the exact byte count.
-template <int D, bool BF16, int PMAX>
+template <int D, bool BF16, int PMAX, bool R8>
 __device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill, const void* q,
                                             const void* k, const void* v, uint8_t* stg,
                                             uint64_t* bar) {
@@ -582,7 +632,8 @@ __device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill
   const int h = head % p.H, b = head / p.H;
   const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
   const bool rows = fill > 0 && fill < p.P;
-  const uint32_t kv_bytes = rows ? (uint32_t)fill * 2 * IO : 0u;
+  constexpr uint32_t RB = D * (R8 ? 1u : (uint32_t)ST::ESZ);   // bytes of a buffered k or v
+  const uint32_t kv_bytes = rows ? (uint32_t)fill * 2 * RB : 0u;
   const uint32_t bytes = 3 * IO + 2 * D + (rows ? kv_bytes + p.ab_stride + p.gram_stride : 0u);
   fence_proxy_async_smem();
   mbar_arrive_expect_tx(bar, bytes);
@@ -591,13 +642,13 @@ __device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill
   tma_load_1d(stg + ST::V, reinterpret_cast<const uint8_t*>(v) + (size_t)head * IO, IO, bar);
   tma_load_1d(stg + ST::SC, rec + code_bytes(D, D, p.bits[h]), 2 * D, bar);
   if (rows) {
-    tma_load_1d(stg + ST::KV, p.kv + (size_t)head * p.P * 2 * IO, kv_bytes, bar);
+    tma_load_1d(stg + ST::KV, p.kv + (size_t)head * p.P * 2 * RB, kv_bytes, bar);
     tma_load_1d(stg + ST::AB, p.ab + (size_t)head * p.ab_stride, p.ab_stride, bar);
     tma_load_1d(stg + ST::G, p.gram + (size_t)head * p.gram_stride, p.gram_stride, bar);
   }
 }
 
-template <int D, bool BF16, int PMAX, bool EXACT, bool ADAPT>
+template <int D, bool BF16, int PMAX, bool EXACT, bool ADAPT, bool R8>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_step_kernel(PoolDev p, const void* __restrict__ q, const void* __restrict__ k,
                        const void* __restrict__ v, const void* __restrict__ alpha,
@@ -623,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp0 < n_heads) {
       const int h0 = head_in_order(p, warp0, sp.b0, sp.nb);
       f_cur = p.fill[h0];
-      if (NS == 2) issue_stage<D, BF16, PMAX>(p, h0, f_cur, q, k, v, stages, &bar[0]);
+      if (NS == 2) issue_stage<D, BF16, PMAX, R8>(p, h0, f_cur, q, k, v, stages, &bar[0]);
       f_nxt = warp0 + W < n_heads ? p.fill[head_in_order(p, warp0 + W, sp.b0, sp.nb)] : 0;
     }
   }
@@ -636,9 +687,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       if (NS == 2) {
         if (nh >= 0)
-          issue_stage<D, BF16, PMAX>(p, nh, f_nxt, q, k, v, stages + (s ^ 1) * ST::BYTES, &bar[s ^ 1]);
+          issue_stage<D, BF16, PMAX, R8>(p, nh, f_nxt, q, k, v, stages + (s ^ 1) * ST::BYTES, &bar[s ^ 1]);
       } else {
-        issue_stage<D, BF16, PMAX>(p, head, f_cur, q, k, v, stages, &bar[0]);
+        issue_stage<D, BF16, PMAX, R8>(p, head, f_cur, q, k, v, stages, &bar[0]);
       }
       if (nh >= 0) {   // the next head's codes on their way into L2
         const int hh = nh % p.H;
@@ -669,9 +720,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int n = nprev + 1;
     if (p.bits[head % p.H] == 4)
-      decode_head<D, BF16, PMAX, 4, EXACT, ADAPT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
+      decode_head<D, BF16, PMAX, 4, EXACT, ADAPT, R8>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
     else
-      decode_head<D, BF16, PMAX, 8, EXACT, ADAPT>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
+      decode_head<D, BF16, PMAX, 8, EXACT, ADAPT, R8>(p, head, n, q, k, v, alpha, beta, o, scr, stg, lane);
   }
 }
 
@@ -688,13 +739,13 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, bool BF16, int PMAX, bool EXACT, bool ADAPT = false>
+template <int D, bool BF16, int PMAX, bool EXACT, bool ADAPT = false, bool R8 = false>
 cudaError_t launch_t(const PoolDev& p, const Span& sp, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
   using ST = Stage<D, BF16, PMAX>;
   const size_t smem = (size_t)kWarpsPerBlock * (ST::N * ST::BYTES + sizeof(WarpScratch<D, ADAPT>) +
                                                 ST::N * sizeof(uint64_t));
-  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX, EXACT, ADAPT>,
+  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D, BF16, PMAX, EXACT, ADAPT, R8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long heads = (long)sp.nb * p.H;
@@ -702,7 +753,7 @@ cudaError_t launch_t(const PoolDev& p, const Span& sp, const void* q, const void
   long blocks = (heads + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const long cap = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 2) * sm_count();
   if (blocks > cap) blocks = cap;
-  decode_step_kernel<D, BF16, PMAX, EXACT, ADAPT><<<(unsigned)blocks, kThreads, smem, st>>>(
+  decode_step_kernel<D, BF16, PMAX, EXACT, ADAPT, R8><<<(unsigned)blocks, kThreads, smem, st>>>(
       p, q, k, v, alpha, beta, o, sp);
   return cudaGetLastError();
 }
@@ -710,6 +761,16 @@ cudaError_t launch_t(const PoolDev& p, const Span& sp, const void* q, const void
 template <int D, bool BF16>
 cudaError_t launch_p(const PoolDev& p, const Span& sp, const void* q, const void* k, const void* v,
                      const void* alpha, const void* beta, float* o, cudaStream_t st) {
+  if (p.row8) {       // E4M3 buffered rows (no commit threshold on such pools)
+    switch (p.P) {
+      case 4: return launch_t<D, BF16, 4, true, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+      case 8: return launch_t<D, BF16, 8, true, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+      case 16: return launch_t<D, BF16, 16, true, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+    }
+    if (p.P < 4) return launch_t<D, BF16, 4, false, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+    if (p.P < 8) return launch_t<D, BF16, 8, false, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+    return launch_t<D, BF16, 16, false, false, true>(p, sp, q, k, v, alpha, beta, o, st);
+  }
   if (p.adaptive) {   // commit threshold set: the period is the buffer's capacity
     if (p.P <= 4) return launch_t<D, BF16, 4, false, true>(p, sp, q, k, v, alpha, beta, o, st);
     if (p.P <= 8) return launch_t<D, BF16, 8, false, true>(p, sp, q, k, v, alpha, beta, o, st);

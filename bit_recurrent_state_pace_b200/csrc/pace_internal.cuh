@@ -34,7 +34,11 @@ struct PoolDev {
   int32_t H4;                         // number of 4-bit heads
   float tau2;                         // commit threshold squared (+inf: fixed period)
   int32_t adaptive;                   // tau2 finite
+  int32_t row8;                       // buffered k, v rows are E4M3 bytes
 };
+
+// Bytes per buffered k or v element.
+__host__ __device__ inline int row_esz(const PoolDev& p) { return p.row8 ? 1 : (p.io == PACE_IO_BF16 ? 2 : 4); }
 
 // A head's buffer is due for a commit: full, or marked by the decode step
 // (which marks only heads holding at least one token).

@@ -56,6 +56,7 @@ pace_status check_desc(const pace_pool_desc* d) {
   for (int h = 0; h < d->num_heads; ++h)
     if (d->head_bits[h] != 4 && d->head_bits[h] != 8) return PACE_ERR_INVALID_ARG;
   if (d->d_k < 1 || d->d_v < 1) return PACE_ERR_INVALID_ARG;
+  if (d->buffer_e4m3 != 0 && d->buffer_e4m3 != 1) return PACE_ERR_INVALID_ARG;
   if (d->d_k != d->d_v) return PACE_ERR_UNSUPPORTED;
   if (d->d_k != 32 && d->d_k != 64 && d->d_k != 128) return PACE_ERR_UNSUPPORTED;
   return PACE_OK;
@@ -73,7 +74,7 @@ pace_status compute_layout(const pace_pool_desc* d, Layout* L) {
   }
   L->slot_stride = round_up(off, 16);
   if (!mul_ok(L->slot_stride, (size_t)d->num_slots, &L->state_bytes)) return PACE_ERR_INVALID_ARG;
-  const size_t esz = (size_t)pace::io_size(d->io_dtype);
+  const size_t esz = d->buffer_e4m3 ? 1 : (size_t)pace::io_size(d->io_dtype);   // buffered k, v
   size_t heads = 0, rows = 0, kv = 0, ab = 0, gram = 0;
   if (!mul_ok((size_t)d->num_slots, (size_t)d->num_heads, &heads)) return PACE_ERR_INVALID_ARG;
   if (!mul_ok(heads, (size_t)d->period, &rows)) return PACE_ERR_INVALID_ARG;
@@ -163,6 +164,7 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
   }
   dv.tau2 = INFINITY;
   dv.adaptive = 0;
+  dv.row8 = desc->buffer_e4m3;
   for (int h = 0; h < desc->num_heads; ++h) {
     dv.rec_off[h] = (uint32_t)L.rec_off[h];
     dv.bits[h] = desc->head_bits[h];
@@ -231,6 +233,7 @@ pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, cons
 
 pace_status pace_set_commit_threshold(pace_pool* pool, float tau) {
   if (!pool || !(tau >= 0.f)) return PACE_ERR_INVALID_ARG;   // NaN fails the comparison
+  if (pool->dev.row8 && std::isfinite(tau)) return PACE_ERR_UNSUPPORTED;
   pool->dev.adaptive = std::isfinite(tau) ? 1 : 0;
   pool->dev.tau2 = pool->dev.adaptive ? tau * tau : INFINITY;
   return PACE_OK;
@@ -370,9 +373,14 @@ pace_status pace_window_step(pace_pool* pool, const void* q, const void* k, cons
   uint8_t* v8 = k8 + round_up(BH * pool->dev.d_k * esz, 256);
   cudaStream_t st = as_stream(stream);
   const pace::Span all{0, pool->dev.B, 0};
-  cudaError_t e = pace::launch_e4m3_round(k, k8, (int64_t)(BH * pool->dev.d_k), pool->dev.io, st);
-  if (e == cudaSuccess) e = pace::launch_e4m3_round(v, v8, (int64_t)(BH * pool->dev.d_v), pool->dev.io, st);
-  if (e == cudaSuccess) e = pace::launch_decode_step(pool->dev, all, q, k8, v8, alpha, beta, o, st);
+  cudaError_t e = cudaSuccess;
+  if (pool->dev.row8) {   // E4M3 rows: the decode rounds k and v as it buffers them
+    e = pace::launch_decode_step(pool->dev, all, q, k, v, alpha, beta, o, st);
+  } else {
+    e = pace::launch_e4m3_round(k, k8, (int64_t)(BH * pool->dev.d_k), pool->dev.io, st);
+    if (e == cudaSuccess) e = pace::launch_e4m3_round(v, v8, (int64_t)(BH * pool->dev.d_v), pool->dev.io, st);
+    if (e == cudaSuccess) e = pace::launch_decode_step(pool->dev, all, q, k8, v8, alpha, beta, o, st);
+  }
   if (e == cudaSuccess) e = pace::launch_window_prepare(pool->dev, st);
   if (e == cudaSuccess) {
     pace::PoolDev one = pool->dev;   // commits the marked heads with their own token count

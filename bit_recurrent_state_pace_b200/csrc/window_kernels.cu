@@ -18,8 +18,7 @@
 //    use, and the commit applies that pair alone (n = 1);
 //  * the remaining S - 1 pairs move down one row, their Gram entries are
 //    recomputed, and fill = S - 1.
-#include <cuda_fp8.h>
-
+#include "e4m3.cuh"
 #include "window.cuh"
 
 namespace pace {
@@ -27,11 +26,6 @@ namespace pace {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-
-__device__ __forceinline__ float e4m3_round(float x) {
-  const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
-  return __half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3)));
-}
 
 // dst[i] = E4M3(src[i]) in the io dtype, for n elements.
 __global__ void e4m3_round_kernel(const void* __restrict__ src, void* __restrict__ dst, int64_t n, int io) {
@@ -58,9 +52,10 @@ __global__ void window_prepare_kernel(PoolDev p, int n_heads) {
   const int head = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   if (head >= n_heads || p.fill[head] != p.P) return;
   const int P = p.P, h = head % p.H, b = head / p.H;
-  const uint8_t* k0 = p.kv + (size_t)head * P * (size_t)(p.d_k + p.d_v) * io_size(p.io);
+  const uint8_t* k0 = p.kv + (size_t)head * P * (size_t)(p.d_k + p.d_v) * row_esz(p);
   float km = 0.f;
-  for (int j = lane; j < p.d_k; j += 32) km = fmaxf(km, fabsf(load_io(k0, j, p.io)));
+  for (int j = lane; j < p.d_k; j += 32)
+    km = fmaxf(km, fabsf(p.row8 ? row_at<true>(k0, j, false) : load_io(k0, j, p.io)));
   km = warp_max(km);
   const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[h];
   const uint16_t* sc = reinterpret_cast<const uint16_t*>(rec + code_bytes(p.d_k, p.d_v, p.bits[h]));
@@ -86,7 +81,7 @@ __global__ void window_shift_kernel(PoolDev p, int n_heads) {
   const int head = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   if (head >= n_heads || p.fill[head] != 0) return;
   const int P = p.P, esz = io_size(p.io);
-  const size_t row = (size_t)(p.d_k + p.d_v) * esz;             // bytes, a multiple of 64
+  const size_t row = (size_t)(p.d_k + p.d_v) * row_esz(p);      // bytes, a multiple of 64
   uint8_t* kv = p.kv + (size_t)head * P * row;
   for (int r = 0; r + 1 < P; ++r) {
     const uint4* src = reinterpret_cast<const uint4*>(kv + (r + 1) * row);
@@ -115,8 +110,11 @@ __global__ void window_shift_kernel(PoolDev p, int n_heads) {
   for (int t = 1; t + 1 < P; ++t)
     for (int s = 0; s < t; ++s) {
       float acc = 0.f;
-      for (int j = lane; j < p.d_k; j += 32)
-        acc = fmaf(load_io(kv + t * row, j, p.io), load_io(kv + s * row, j, p.io), acc);
+      for (int j = lane; j < p.d_k; j += 32) {
+        const float a = p.row8 ? row_at<true>(kv + t * row, j, false) : load_io(kv + t * row, j, p.io);
+        const float c = p.row8 ? row_at<true>(kv + s * row, j, false) : load_io(kv + s * row, j, p.io);
+        acc = fmaf(a, c, acc);
+      }
 #pragma unroll
       for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
       if (lane == 0) g[t * P + s] = acc;

@@ -76,6 +76,8 @@ typedef struct {
   int32_t scale_axis;         /* pace_scale_axis */
   int32_t io_dtype;           /* pace_io_dtype */
   const uint8_t* head_bits;   /* host array [num_heads], each 4 or 8 ([P4] TL;DR (3)) */
+  int32_t buffer_e4m3;        /* 0: buffered k, v in io_dtype; 1: as FP8 E4M3 bytes (the
+                                 pure-write window's pairs, see pace_window_step) */
 } pace_pool_desc;
 
 /*
@@ -90,7 +92,9 @@ typedef struct {
  *          record padded to 16 bytes.
  * buffer : the token buffer ([P2] "Periodic Rounding"; [P4] flowchart "Small
  *          buffer, last few tokens"): region KV = [B][H][P][d_k + d_v]
- *          io_dtype elements (row = k then v of one buffered token), then at
+ *          io_dtype elements (row = k then v of one buffered token; one E4M3
+ *          byte per element when buffer_e4m3 is set, the token's k and v then
+ *          rounded to E4M3 as they are buffered and used), then at
  *          byte offset round_up(size(KV), 256) region AB: [B][H] blocks of
  *          round_up(2*P*io_size, 16) bytes, each [P][2] io_dtype elements
  *          (alpha, beta); then at the next 256-byte boundary region G: [B][H]

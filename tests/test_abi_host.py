@@ -72,6 +72,18 @@ def test_descriptor_validation(kw, status):
     assert e.value.status == status
 
 
+def test_e4m3_buffer_layout():
+    import bit_recurrent_state_pace_b200 as pace
+    bits = [8] * 12 + [4] * 36
+    st, buf, _ = pace.pace_pool_bytes(4096, 48, 128, 128, 8, 0, 0, bits, 1)
+    st0, buf0, _ = pace.pace_pool_bytes(4096, 48, 128, 128, 8, 0, 0, bits, 0)
+    # k, v rows at one byte per element; gates and Gram cache unchanged
+    assert st == st0 and buf0 - buf == 4096 * 48 * 8 * 256
+    with pytest.raises(pace.PaceError) as e:
+        pace.pace_pool_bytes(2, 4, 128, 128, 8, 0, 0, [4] * 4, 2)
+    assert e.value.status == 1
+
+
 def test_status_strings():
     import bit_recurrent_state_pace_b200 as pace
     assert pace.pace_status_string(0) == "PACE_OK"

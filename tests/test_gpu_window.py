@@ -9,7 +9,8 @@ stored history and the pairs in its window; it then
   * when the window was full, merges the oldest pair into the history and
     encodes it, and the GPU's new history must match (ties only, R15).
 A window of one step must be the period-one path on E4M3-rounded inputs,
-bit for bit.
+bit for bit.  The pairs are held either as E4M3 bytes (a pool created with
+buffer_e4m3) or as E4M3 values in the io dtype.
 """
 import numpy as np
 import pytest
@@ -27,6 +28,19 @@ def _pace():
     return pace
 
 
+def _e4m3_table():
+    """Value of every E4M3 byte, decoded from its fields (NaN for S.1111.111)."""
+    t = np.empty(256)
+    for c in range(256):
+        s, E, m = c >> 7, (c >> 3) & 15, c & 7
+        v = np.nan if (E == 15 and m == 7) else (m * 2.0 ** -9 if E == 0 else (1 + m / 8) * 2.0 ** (E - 7))
+        t[c] = -v if s else v
+    return t
+
+
+E4M3 = _e4m3_table()
+
+
 def _window_rows(pool, w, n):
     """Host copies of the first n window pairs of every head: k, v [N][n][d],
     alpha, beta [N][n] (float64), read through the documented buffer layout."""
@@ -34,8 +48,12 @@ def _window_rows(pool, w, n):
     dt = torch.bfloat16 if esz == 2 else torch.float32
     BH, P, D = w.B * w.H, w.P, w.d_k
     ru = lambda x, a: (x + a - 1) // a * a
-    kv_bytes = BH * P * (w.d_k + w.d_v) * esz
-    kv = pool.buffer[:kv_bytes].view(dt).view(BH, P, w.d_k + w.d_v).to(torch.float64).cpu().numpy()
+    resz = 1 if pool.buffer_e4m3 else esz
+    kv_bytes = BH * P * (w.d_k + w.d_v) * resz
+    if pool.buffer_e4m3:
+        kv = E4M3[pool.buffer[:kv_bytes].cpu().numpy().astype(np.int64)].reshape(BH, P, w.d_k + w.d_v)
+    else:
+        kv = pool.buffer[:kv_bytes].view(dt).view(BH, P, w.d_k + w.d_v).to(torch.float64).cpu().numpy()
     ab_stride = ru(2 * P * esz, 16)
     ab_off = ru(kv_bytes, 256)
     ab = pool.buffer[ab_off:ab_off + BH * ab_stride].view(BH, ab_stride)[:, :2 * P * esz]
@@ -43,13 +61,14 @@ def _window_rows(pool, w, n):
     return kv[:, :n, :D], kv[:, :n, D:], ab[:, :n, 0], ab[:, :n, 1]
 
 
-def _run(w, T, seed=0):
+def _run(w, T, seed=0, e4m3_rows=False):
     pace = _pace()
     bits = pace_synth.head_bits(w, seed)
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     S0 = pace_synth.random_state(len(heads), w.d_v, w.d_k, seed=seed).numpy()
     state, _ = orc.PoolState.from_fp32(S0, [bits[h] for _, h in heads], w.axis)
-    pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype)
+    pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype,
+                         buffer_e4m3=e4m3_rows)
     pu.load_state(pool, heads, state)
     hbits = [bits[h] for _, h in heads]
     worst, merges = 0.0, 0
@@ -94,17 +113,48 @@ def _run(w, T, seed=0):
     return worst, merges
 
 
+@pytest.mark.parametrize("e4m3_rows", [True, False])
 @pytest.mark.parametrize("name,over", [
     ("mixed_4_8", {}),
     ("mixed_4_8", dict(axis="row")),
     ("gdn_layer_4b", dict(d_k=64, d_v=64, P=5, io_dtype="f32", outliers=False)),
     ("mixed_4_8", dict(d_k=32, d_v=32, P=16)),
 ])
-def test_window_against_oracle(name, over):
+def test_window_against_oracle(name, over, e4m3_rows):
+    """The window's pairs as E4M3 bytes (the pool's buffer_e4m3 layout) or as
+    E4M3 values in the io dtype."""
     w = pace_synth.workload(name, B=2, H=4, **over)
-    worst, merges = _run(w, T=2 * w.P + 3)
-    print(name, over, "worst", worst, "merges", merges)
+    worst, merges = _run(w, T=2 * w.P + 3, e4m3_rows=e4m3_rows)
+    print(name, over, "e4m3 rows" if e4m3_rows else "io rows", "worst", worst, "merges", merges)
     assert merges == w.P + 4
+
+
+def test_period_with_an_e4m3_buffer_against_oracle():
+    """pace_decode_step / pace_commit_period on a pool whose buffer holds E4M3
+    bytes: one teacher-forced period of the oracle on E4M3-rounded k, v."""
+    pace = _pace()
+    w = pace_synth.workload("mixed_4_8", B=2, H=4)
+    bits = pace_synth.head_bits(w, 0)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    S0 = pace_synth.random_state(len(heads), w.d_v, w.d_k, seed=2).numpy()
+    state, _ = orc.PoolState.from_fp32(S0, [bits[h] for _, h in heads], w.axis)
+    pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype,
+                         buffer_e4m3=True)
+    pu.load_state(pool, heads, state)
+    toks, outs = [], []
+    for t in range(w.P):
+        x = pace_synth.token_inputs(w, t, seed=2, device="cuda")
+        outs.append(pool.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"]).cpu().numpy()
+                    .reshape(len(heads), w.d_v))
+        tok = pu.host_tokens(x, heads)
+        toks.append(dict(tok, k=orc.e4m3(tok["k"]), v=orc.e4m3(tok["v"])))
+    pool.commit_period()
+    assert pool.status() == 0
+    o_ref, S_end, committed, _ = orc.period_reference(state, toks, w.P)
+    for n in range(w.P):
+        assert orc.relative_error(outs[n], o_ref[n]).max() <= pu.O_TOL, n
+    gc, gs = pu.read_state(pool, heads)
+    pu.judge_commit(gc, gs, committed, S_end, w.axis)
 
 
 def test_window_of_one_is_period_one_on_rounded_inputs():
@@ -134,6 +184,10 @@ def test_window_of_one_is_period_one_on_rounded_inputs():
 def test_window_rejects_a_threshold_pool():
     pace = _pace()
     w = pace_synth.workload("tiny")
+    e = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, pace_synth.head_bits(w, 0), io=w.io_dtype,
+                      buffer_e4m3=True)
+    with pytest.raises(pace.PaceError):
+        e.set_commit_threshold(1.0)
     pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, pace_synth.head_bits(w, 0), io=w.io_dtype)
     pool.set_commit_threshold(1.0)
     x = pace_synth.token_inputs(w, 0, device="cuda")
