@@ -178,7 +178,8 @@ pace_status pace_decode_step(pace_pool* pool, const void* q, const void* k, cons
  * PACE_FILL_COMMIT); pace_commit_period then commits it with its n tokens,
  * and a decode step on a marked head is skipped like one on a full buffer.
  * tau = +inf (the default) is the fixed period P; tau = 0 commits after
- * every token.  A negative or NaN tau is PACE_ERR_INVALID_ARG.  Host-only:
+ * every token.  A negative or NaN tau is PACE_ERR_INVALID_ARG; a finite tau
+ * on a pool with buffer_e4m3 set is PACE_ERR_UNSUPPORTED.  Host-only:
  * applies to launches enqueued after the call.
  */
 pace_status pace_set_commit_threshold(pace_pool* pool, float tau);
