@@ -55,6 +55,29 @@ def test_host_path_matches_device_calls_bit_for_bit(name, axis):
     assert torch.equal(dev.fill(), host.fill())
 
 
+def test_host_path_with_a_commit_threshold():
+    """With a commit threshold the host path commits the heads each step marks,
+    exactly as the device-path calls do."""
+    w = pace_synth.workload("mixed_4_8", B=6)
+    bits = pace_synth.head_bits(w, 0)
+    S = pace_synth.random_state(w.B * w.H, w.d_v, w.d_k, seed=8, device="cuda").view(
+        w.B, w.H, w.d_v, w.d_k)
+    dev, host = _pool(w, bits, S), _pool(w, bits, S)
+    for pool in (dev, host):
+        pool.set_commit_threshold(4.0)
+    T = 2 * w.P + 1
+    h = _host_tokens(w, 0, T)
+    o_dev = torch.empty(T, w.B, w.H, w.d_v, device="cuda")
+    _device_run(dev, w, h, o_dev)
+    o_host = torch.empty(T, w.B, w.H, w.d_v).pin_memory()
+    host.decode_host(h["q"], h["k"], h["v"], h["alpha"], h["beta"], o_host)
+    torch.cuda.synchronize()
+    assert torch.equal(o_dev.cpu(), o_host)
+    assert torch.equal(dev.state, host.state)
+    assert torch.equal(dev.fill(), host.fill())
+    assert dev.status() == 0 and host.status() == 0
+
+
 def test_host_path_without_outputs_still_advances_the_pool():
     w = pace_synth.workload("mixed_4_8", B=8)
     bits = pace_synth.head_bits(w, 0)
