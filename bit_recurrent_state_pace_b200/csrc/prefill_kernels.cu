@@ -45,8 +45,10 @@ template <int D, bool BF16>
 struct alignas(16) PSmem {
   using C = PCfg<D, BF16>;
   // chunk rows k [0], q [1], v [2] in the io dtype, double-buffered: chunk
-  // c + 1 arrives by asynchronous copies while chunk c computes
-  uint8_t raw[2][3][CH][D * (BF16 ? 2 : 4)];
+  // c + 1 arrives by asynchronous copies while chunk c computes.  Rows sit
+  // 16 bytes past a multiple of 128, so the same channel of different
+  // tokens falls in different banks when the operand tables gather it.
+  uint8_t raw[2][3][CH][D * (BF16 ? 2 : 4) + 16];
   float abuf[2][2][CH];               // [buffer][alpha, beta][token]
   uint2 bx[C::NKX][C::KS][8][4];      // K / Q B fragments [tile][ks][g][t]
   uint2 bkf[C::NT][C::KU][8][4];      // update B fragments [tile][u][g][t]
