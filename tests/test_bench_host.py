@@ -1,0 +1,41 @@
+"""bench.py on the CPU: the reference arm's JSON line, and the ncu records in
+profiles/ that the GPU line's roofline `traffic` is read from."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench_module():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_reference_arm_prints_the_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "1"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "impl",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_profiles_hold_traffic_for_the_current_kernel_sources():
+    """Every ncu traffic record the roofline reads belongs to the kernel sources
+    as they are: a change to a kernel without a new capture fails here."""
+    bench = _bench_module()
+    for kernel in ("decode_step", "commit"):
+        digest = bench.kernel_source_digest(kernel)
+        traffic = bench.ncu_traffic(kernel, digest)
+        assert traffic is not None and traffic > 0, (kernel, digest)
