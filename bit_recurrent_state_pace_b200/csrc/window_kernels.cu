@@ -75,51 +75,84 @@ __global__ void window_prepare_kernel(PoolDev p, int n_heads) {
 
 // One warp per head.  A head whose oldest pair was just merged (fill 0 after
 // the commit): rows 1..P-1 and their gates move down one, the Gram entries of
-// the remaining pairs are recomputed, fill = P - 1.
+// the remaining pairs are recomputed, fill = P - 1.  The moves go four rows
+// at a time (loads in flight together, then the stores); the keys of the
+// remaining pairs are read once into registers (EPL channels per lane) and
+// every Gram entry is a register dot product and a warp sum.
+template <int D, int PMAX>
 __global__ void window_shift_kernel(PoolDev p, int n_heads) {
+  constexpr int EPL = D / 32;
   const int lane = threadIdx.x & 31;
   const int head = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   if (head >= n_heads || p.fill[head] != 0) return;
-  const int P = p.P, esz = io_size(p.io);
+  const int P = p.P;
   const size_t row = (size_t)(p.d_k + p.d_v) * row_esz(p);      // bytes, a multiple of 64
+  const int n16 = (int)(row / 16);                              // <= 64
   uint8_t* kv = p.kv + (size_t)head * P * row;
-  for (int r = 0; r + 1 < P; ++r) {
-    const uint4* src = reinterpret_cast<const uint4*>(kv + (r + 1) * row);
-    uint4* dst = reinterpret_cast<uint4*>(kv + r * row);
-    const int n16 = (int)(row / 16);
-    uint4 tmp[8];                                               // row <= 128 x 16 bytes
+  for (int r0 = 0; r0 + 1 < P; r0 += 4) {
+    uint4 tmp[4][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (lane + 32 * i < n16) tmp[i] = src[lane + 32 * i];
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (r0 + rr + 1 < P && lane + 32 * i < n16)
+          tmp[rr][i] = reinterpret_cast<const uint4*>(kv + (r0 + rr + 1) * row)[lane + 32 * i];
     __syncwarp();
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (lane + 32 * i < n16) dst[lane + 32 * i] = tmp[i];
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (r0 + rr + 1 < P && lane + 32 * i < n16)
+          reinterpret_cast<uint4*>(kv + (r0 + rr) * row)[lane + 32 * i] = tmp[rr][i];
     __syncwarp();
   }
-  uint8_t* ab = p.ab + (size_t)head * p.ab_stride;
-  if (lane == 0) {
-    for (int e = 0; e + 2 < 2 * P; ++e) {                        // [P][2] io elements
-      if (esz == 2) reinterpret_cast<uint16_t*>(ab)[e] = reinterpret_cast<uint16_t*>(ab)[e + 2];
-      else reinterpret_cast<float*>(ab)[e] = reinterpret_cast<float*>(ab)[e + 2];
+  {
+    uint8_t* ab = p.ab + (size_t)head * p.ab_stride;            // [P][2] io elements
+    const bool mv = lane + 2 < 2 * P;
+    float x = 0.f;
+    if (mv) x = load_io(ab, lane + 2, p.io);
+    __syncwarp();
+    if (mv) {
+      if (p.io == PACE_IO_BF16) reinterpret_cast<uint16_t*>(ab)[lane] = float_to_bf16_bits_rn(x);   // exact
+      else reinterpret_cast<float*>(ab)[lane] = x;
     }
   }
   __syncwarp();
   // Gram entries G[t][s] = k_t . k_s of the remaining pairs, s < t < P - 1
-  float* g = reinterpret_cast<float*>(p.gram + (size_t)head * p.gram_stride);
-  for (int t = 1; t + 1 < P; ++t)
-    for (int s = 0; s < t; ++s) {
-      float acc = 0.f;
-      for (int j = lane; j < p.d_k; j += 32) {
-        const float a = p.row8 ? row_at<true>(kv + t * row, j, false) : load_io(kv + t * row, j, p.io);
-        const float c = p.row8 ? row_at<true>(kv + s * row, j, false) : load_io(kv + s * row, j, p.io);
-        acc = fmaf(a, c, acc);
-      }
+  float kr[PMAX][EPL];
 #pragma unroll
-      for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
-      if (lane == 0) g[t * P + s] = acc;
+  for (int t = 0; t < PMAX; ++t)
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int j = EPL * lane + e;
+      kr[t][e] = t + 1 < P ? (p.row8 ? row_at<true>(kv + t * row, j, false) : load_io(kv + t * row, j, p.io))
+                           : 0.f;
+    }
+  float* g = reinterpret_cast<float*>(p.gram + (size_t)head * p.gram_stride);
+#pragma unroll
+  for (int t = 1; t < PMAX; ++t)
+#pragma unroll
+    for (int s = 0; s < t; ++s) {
+      if (t + 1 < P) {
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc = fmaf(kr[t][e], kr[s][e], acc);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
+        if (lane == 0) g[t * P + s] = acc;
+      }
     }
   if (lane == 0) p.fill[head] = P - 1;
+}
+
+template <int D>
+cudaError_t launch_shift_d(const PoolDev& p, cudaStream_t st) {
+  const int n = p.B * p.H;
+  const unsigned blocks = (unsigned)((n + 7) / 8);
+  if (p.P <= 4) window_shift_kernel<D, 4><<<blocks, 256, 0, st>>>(p, n);
+  else if (p.P <= 8) window_shift_kernel<D, 8><<<blocks, 256, 0, st>>>(p, n);
+  else window_shift_kernel<D, 16><<<blocks, 256, 0, st>>>(p, n);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -139,9 +172,12 @@ cudaError_t launch_window_prepare(const PoolDev& p, cudaStream_t st) {
 }
 
 cudaError_t launch_window_shift(const PoolDev& p, cudaStream_t st) {
-  const int n = p.B * p.H;
-  window_shift_kernel<<<(unsigned)((n + 7) / 8), 256, 0, st>>>(p, n);
-  return cudaGetLastError();
+  switch (p.d_k) {
+    case 32: return launch_shift_d<32>(p, st);
+    case 64: return launch_shift_d<64>(p, st);
+    case 128: return launch_shift_d<128>(p, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace pace
