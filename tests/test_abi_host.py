@@ -89,3 +89,19 @@ def test_status_strings():
     assert pace.pace_status_string(0) == "PACE_OK"
     assert pace.pace_status_string(3) == "PACE_ERR_CUDA"
     assert pace.pace_version()
+
+
+def test_binding_constants_match_the_header():
+    """Every #define and enum value of include/pace.h that the binding
+    mirrors has the same value there."""
+    import bit_recurrent_state_pace_b200 as pace
+    text = open(os.path.join(ROOT, "include", "pace.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    values = {m.group(1): int(m.group(2), 0)
+              for m in re.finditer(r"#define\s+(PACE_\w+)\s+(0x[0-9a-fA-F]+|\d+)u?", text)}
+    for m in re.finditer(r"(PACE_[A-Z0-9_]+)\s*=\s*(\d+)", text):
+        values[m.group(1)] = int(m.group(2))
+    mirrored = [n for n in values if hasattr(pace, n)]
+    assert len(mirrored) >= 10, mirrored
+    for n in mirrored:
+        assert getattr(pace, n) == values[n], (n, getattr(pace, n), values[n])
