@@ -27,6 +27,7 @@ __all__ = [
     "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
     "pace_select_head_bits", "pace_prefill", "pace_prefill_range", "pace_host_staging_bytes",
     "pace_decode_host", "pace_set_commit_threshold", "pace_window_scratch_bytes", "pace_window_step",
+    "pace_window_step_static", "PACE_WINDOW_STATIC_SCRATCH_BYTES",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -41,6 +42,7 @@ PACE_FLAG_SCALE_OVERFLOW = 0x2
 PACE_FLAG_BUFFER_FULL = 0x4
 PACE_FLAG_TIMEOUT = 0x8
 PACE_FILL_COMMIT = 0x100
+PACE_WINDOW_STATIC_SCRATCH_BYTES = 8 << 20
 PACE_OK, PACE_ERR_DEVICE_FLAGS = 0, 4
 
 
@@ -82,6 +84,7 @@ def _load():
         "pace_set_commit_threshold": [P, ctypes.c_float],
         "pace_window_scratch_bytes": [P, Sp],
         "pace_window_step": [P, P, P, P, P, P, F32p, P, P],
+        "pace_window_step_static": [P, P, P, P, P, P, F32p, P],
         "pace_decode_host": [P, I32, P, P, P, P, P, P, P, P, P, P],
         "pace_prefill_range": [P, I32, I32, I64, P, P, P, P, P, F32p, P],
         "pace_select_head_bits": [P, I32, I32, P],
@@ -200,6 +203,12 @@ def pace_window_scratch_bytes(handle: int) -> int:
 def pace_window_step(handle: int, q, k, v, alpha, beta, o, scratch, stream=None) -> None:
     _check("pace_window_step", lib.pace_window_step(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                                                     _ptr(beta), _ptr(o), _ptr(scratch), _stream(stream)))
+
+
+def pace_window_step_static(handle: int, q, k, v, alpha, beta, o, stream=None) -> None:
+    """pace_window_step with the library's own device scratch (no allocation)."""
+    _check("pace_window_step_static", lib.pace_window_step_static(
+        handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)))
 
 
 def pace_set_commit_threshold(handle: int, tau: float) -> None:

@@ -312,6 +312,33 @@ pace_status pace_window_step(pace_pool* pool, const void* q, const void* k, cons
                              void* stream);
 
 /*
+ * pace_window_step without caller scratch.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory
+ * themselves -- e.g. a plugin inside an inference engine whose allocator owns
+ * the whole device budget and hands out only the tensors of a call's inputs
+ * and outputs, or a hot loop that must not call cudaMalloc, which can
+ * synchronise the device.  It allocates nothing: the scratch for the rounded
+ * k and v is a device array of PACE_WINDOW_STATIC_SCRATCH_BYTES bytes inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.
+ *  - Same arguments, results and errors as pace_window_step, minus
+ *    d_scratch.
+ *  - A pool whose pace_window_scratch_bytes exceeds
+ *    PACE_WINDOW_STATIC_SCRATCH_BYTES is PACE_ERR_UNSUPPORTED (nothing is
+ *    launched); use pace_window_step for it.
+ *  - The first call on a device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress; PACE_ERR_CUDA if that
+ *    fails).  Make that first call before any stream capture.
+ *  - Every call on a device shares the one array.  Calls whose work overlaps
+ *    on the GPU (two streams, or two pools) race on it: order them, e.g. on
+ *    one stream.  Nothing in the array needs clearing between calls: each
+ *    call overwrites what it reads.
+ */
+#define PACE_WINDOW_STATIC_SCRATCH_BYTES 8388608u   /* 8 MiB */
+pace_status pace_window_step_static(pace_pool* pool, const void* q, const void* k, const void* v,
+                                    const void* alpha, const void* beta, float* o, void* stream);
+
+/*
  * Chunked fp32 prefill (the chunked prefill kernels that [P2] "Periodic
  * Rounding" cites; [P4] flowchart "State update, chunked, high precision").
  * For every head of the slots (all of them, or [slot_begin, slot_begin +
