@@ -291,6 +291,33 @@ def check_pack_roundtrip(pack_codes, unpack_codes, seed=0):
     assert pack_codes(np.array([[1, -2]], np.int8), 4).tolist() == [[0xE1]]
 
 
+def check_commit_ratios(commit_ratios):
+    """x / sf of the period-end state, worked by hand on a 2 x 3 state
+    (d_v != d_k, so a scale vector expanded on the wrong axis cannot
+    broadcast) and on a 2 x 2 state with distinct scales (where it can, and
+    gives other numbers).  The entry 1.25 - 2^-30 rounds to 1.25 in fp32
+    ("PACE: A New 4-Bit ...", section "Channel-Aligned Encoding": the state is
+    encoded from its fp32 value), so with sf = 0.5 its ratio is the tie 2.5
+    exactly; in fp64 it would sit 2^-29 below the tie."""
+    S = np.array([[1.5, -3.0, 0.75],
+                  [1.25 - 2.0 ** -30, 0.0, -7.0]], dtype=np.float64)
+    # COL: one scale per key channel j (columns)
+    r = commit_ratios(S, np.array([0.5, 1.0, 0.25], np.float16), "col")
+    assert r.shape == (2, 3)
+    assert r.tolist() == [[3.0, -3.0, 3.0], [2.5, 0.0, -28.0]], r.tolist()
+    # ROW: one scale per value channel i (rows)
+    r = commit_ratios(S, np.array([0.25, 0.375], np.float16), "row")
+    assert r.tolist() == [[6.0, -12.0, 3.0], [10.0 / 3.0, 0.0, -56.0 / 3.0]], r.tolist()
+    # square state, scales 1 and 4: COL divides column 1 by 4, ROW row 1
+    S2 = np.array([[8.0, 8.0], [-2.0, 6.0]])
+    sc = np.array([1.0, 4.0], np.float16)
+    assert commit_ratios(S2, sc, "col").tolist() == [[8.0, 2.0], [-2.0, 1.5]]
+    assert commit_ratios(S2, sc, "row").tolist() == [[8.0, 8.0], [-0.5, 1.5]]
+    # scales are read as the fp16 values stored in the record
+    r = commit_ratios(np.array([[0.5]]), np.array([0.1], np.float16), "col")
+    assert r.tolist() == [[0.5 / (1638.0 / 16384.0)]], r.tolist()
+
+
 # --------------------------------------------------------------------------
 # recurrence checks
 # --------------------------------------------------------------------------

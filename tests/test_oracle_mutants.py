@@ -171,6 +171,32 @@ def test_pack_mutant_is_caught():
     assert _fails(ck.check_encoder_golden, orc.quantize, pack_swapped)
 
 
+# ---------------- tie-checker mutants ----------------
+
+def _ratios_factory(kind):
+    def commit_ratios(S_fp64, scales, axis):
+        S = np.asarray(S_fp64, dtype=np.float64)
+        if kind != "no_fp32_cast":
+            S = S.astype(np.float32).astype(np.float64)
+        sf = np.asarray(scales, dtype=np.float16).astype(np.float64)
+        group = -2 if axis == "col" else -1
+        if kind == "axis_swapped":
+            group = -1 if axis == "col" else -2
+        sf = np.expand_dims(sf, group)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            return S / sf
+    return commit_ratios
+
+
+@pytest.mark.parametrize("kind", ["no_fp32_cast", "axis_swapped"])
+def test_commit_ratios_mutant_is_caught(kind):
+    assert _fails(ck.check_commit_ratios, _ratios_factory(kind)), kind
+
+
+def test_commit_ratios_unmutated_copy_passes():
+    ck.check_commit_ratios(_ratios_factory("none"))
+
+
 # ---------------- adaptive-period mutants ----------------
 
 def _norm_factory(kind):

@@ -34,6 +34,10 @@ def test_pack_roundtrip_and_nibble_order():
     ck.check_pack_roundtrip(orc.pack_codes, orc.unpack_codes)
 
 
+def test_commit_ratios_hand_worked():
+    ck.check_commit_ratios(orc.commit_ratios)
+
+
 def test_gdn_golden_two_tokens():
     ck.check_gdn_golden(orc.gdn_step)
 
