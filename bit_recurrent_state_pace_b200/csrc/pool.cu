@@ -4,11 +4,15 @@
 
 #include <cmath>
 
+#include "commit_tc.cuh"
 #include "pace_internal.cuh"
 #include "window.cuh"
 
 struct pace_pool {
   pace::PoolDev dev;
+  // tensor maps of the state region for the tensor-memory commit (d = 128)
+  pace::CommitMaps maps;
+  bool maps_ok = false;
   pace_pool_desc desc;
   size_t state_bytes, buffer_bytes, aux_bytes, kv_bytes;
   size_t rec_bytes[PACE_MAX_HEADS];
@@ -30,6 +34,14 @@ inline pace_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return PACE_OK;
   (void)cudaGetLastError();  // clear a non-sticky error so later calls start clean
   return PACE_ERR_CUDA;
+}
+
+// Period commit of the heads due in a span: the tensor-memory kernel for the
+// shapes it is built for, the mma.sync kernel otherwise.
+inline cudaError_t commit_launch(const pace_pool* pool, const pace::PoolDev& dev, const pace::Span& sp,
+                                 cudaStream_t st) {
+  if (pool->maps_ok && pace::commit_tc_supported(dev)) return pace::launch_commit_tc(dev, sp, pool->maps, st);
+  return pace::launch_commit(dev, sp, st);
 }
 
 inline bool mul_ok(size_t a, size_t b, size_t* out) {
@@ -170,6 +182,8 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
     dv.bits[h] = desc->head_bits[h];
     p->rec_bytes[h] = L.rec_bytes[h];
   }
+  if (desc->d_k == 128 && desc->d_v == 128)
+    p->maps_ok = pace::make_commit_maps(dv.state, L.state_bytes, &p->maps);
   cudaError_t e = cudaMemsetAsync(d_aux, 0, L.aux_bytes, as_stream(stream));
   if (e != cudaSuccess) {
     delete p;
@@ -243,7 +257,7 @@ pace_status pace_commit_period_range(pace_pool* pool, int32_t slot_begin, int32_
                                      int32_t blocks_per_sm, void* stream) {
   if (!pool || !span_ok(pool, slot_begin, slot_count, blocks_per_sm)) return PACE_ERR_INVALID_ARG;
   const pace::Span sp{slot_begin, slot_count, blocks_per_sm};
-  return from_cuda(pace::launch_commit(pool->dev, sp, as_stream(stream)));
+  return from_cuda(commit_launch(pool, pool->dev, sp, as_stream(stream)));
 }
 
 pace_status pace_prefill_range(pace_pool* pool, int32_t slot_begin, int32_t slot_count,
@@ -339,7 +353,7 @@ pace_status pace_decode_host(pace_pool* pool, int32_t n_tokens, const void* h_q,
     const pace::Span all{0, pool->dev.B, 0};
     e = pace::launch_decode_step(pool->dev, all, base + hs.q, base + hs.k, base + hs.v, base + hs.a,
                                  base + hs.b, reinterpret_cast<float*>(base + hs.o), cs);
-    if (e == cudaSuccess) e = pace::launch_commit(pool->dev, all, cs);   // heads whose buffer filled
+    if (e == cudaSuccess) e = commit_launch(pool, pool->dev, all, cs);   // heads whose buffer filled
     if (e == cudaSuccess) e = cudaEventRecord(computed[sl], cs);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(hs_out, computed[sl], 0);
     if (e == cudaSuccess && h_o)
@@ -385,7 +399,7 @@ pace_status pace_window_step(pace_pool* pool, const void* q, const void* k, cons
   if (e == cudaSuccess) {
     pace::PoolDev one = pool->dev;   // commits the marked heads with their own token count
     one.adaptive = 1;
-    e = pace::launch_commit(one, all, st);
+    e = commit_launch(pool, one, all, st);
   }
   if (e == cudaSuccess) e = pace::launch_window_shift(pool->dev, st);
   return from_cuda(e);
