@@ -27,7 +27,8 @@ __all__ = [
     "pace_decode_step_range", "pace_commit_period_range", "pace_decay_rates",
     "pace_select_head_bits", "pace_prefill", "pace_prefill_range", "pace_host_staging_bytes",
     "pace_decode_host", "pace_set_commit_threshold", "pace_window_scratch_bytes", "pace_window_step",
-    "pace_window_step_static", "PACE_WINDOW_STATIC_SCRATCH_BYTES",
+    "pace_window_step_static", "PACE_WINDOW_STATIC_SCRATCH_BYTES", "pace_set_commit_engine",
+    "PACE_COMMIT_MMA", "PACE_COMMIT_TCGEN05",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -43,6 +44,7 @@ PACE_FLAG_BUFFER_FULL = 0x4
 PACE_FLAG_TIMEOUT = 0x8
 PACE_FILL_COMMIT = 0x100
 PACE_WINDOW_STATIC_SCRATCH_BYTES = 8 << 20
+PACE_COMMIT_MMA, PACE_COMMIT_TCGEN05 = 0, 1
 PACE_OK, PACE_ERR_DEVICE_FLAGS = 0, 4
 
 
@@ -82,6 +84,7 @@ def _load():
         "pace_prefill": [P, I64, P, P, P, P, P, F32p, P],
         "pace_host_staging_bytes": [P, Sp],
         "pace_set_commit_threshold": [P, ctypes.c_float],
+        "pace_set_commit_engine": [P, I32],
         "pace_window_scratch_bytes": [P, Sp],
         "pace_window_step": [P, P, P, P, P, P, F32p, P, P],
         "pace_window_step_static": [P, P, P, P, P, P, F32p, P],
@@ -213,6 +216,10 @@ def pace_window_step_static(handle: int, q, k, v, alpha, beta, o, stream=None) -
 
 def pace_set_commit_threshold(handle: int, tau: float) -> None:
     _check("pace_set_commit_threshold", lib.pace_set_commit_threshold(handle, float(tau)))
+
+
+def pace_set_commit_engine(handle: int, engine: int) -> None:
+    _check("pace_set_commit_engine", lib.pace_set_commit_engine(handle, int(engine)))
 
 
 def pace_host_staging_bytes(handle: int) -> int:
@@ -409,6 +416,10 @@ class PacePool:
             o = torch.empty(self.B, self.H, self.d_v, dtype=torch.float32, device=self.state.device)
         pace_window_step(self.handle, q, k, v, alpha, beta, o, self._wscratch, stream)
         return o
+
+    def set_commit_engine(self, engine: int) -> None:
+        """PACE_COMMIT_MMA (default) or PACE_COMMIT_TCGEN05 for later commits."""
+        pace_set_commit_engine(self.handle, engine)
 
     def set_commit_threshold(self, tau: float) -> None:
         """Adaptive period: a head is committed early once the Frobenius norm of

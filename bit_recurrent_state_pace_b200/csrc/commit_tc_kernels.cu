@@ -33,6 +33,8 @@
 //    (scales).
 // Every wait is bounded; a wait that gives up sets PACE_FLAG_TIMEOUT and the
 // CTA drains its tensor work, frees TMEM and returns.
+#include <type_traits>
+
 #include "commit_tc.cuh"
 #include "e4m3.cuh"
 #include "tc.cuh"
@@ -64,7 +66,7 @@ struct TcCfg {
   static constexpr int FIXED = 2 * (TILE + STG + BXB + 2 * AUB) + 4096;
   static constexpr int NST_FIT = (kSmemLimit - 1024 - FIXED) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;  // staged heads
-  static constexpr int THREADS = 14 * 32;                 // producer, MMA, 4 converter, 8 epilogue warps
+  static constexpr int THREADS = 10 * 32;                 // producer, MMA, 4 converter, 4 epilogue warps
   static constexpr int CONV0 = 2, EPI0 = 6;               // first converter / epilogue warp
 };
 
@@ -78,10 +80,11 @@ struct alignas(1024) TcSmem {
   uint8_t bu[2][C::AUB];               // update B (U^, K-major): [KU/16][16][2][8][8], no swizzle
   uint8_t stage[C::NST][C::STAGE];     // record | rows | factor block
   __half ident[256];                   // 16 x 16 identity, K-major, no swizzle
-  float fj[2][128];                    // epilogue factors gamma_n s_j 2^e, by tile position
-  float amax_x[2][128];                // per-column partial maxima of the two column halves
+  // per-head values handed from the converters to the MMA warp and the
+  // epilogue, in a ring of four (the head k + 4 reuses the slot of head k)
+  float fj[4][128];                    // epilogue factors gamma_n s_j 2^e, by tile position
+  int meta_head[4], meta_e[4], meta_bits[4];
   float red[2][4];                     // converter maxima of |U^| (two heads alternate)
-  int meta_head[2], meta_n[2], meta_e[2];
   int stage_head[C::NST], stage_n[C::NST];
   uint64_t stage_full[C::NST], stage_empty[C::NST];
   uint64_t tile_full[2], x_full[2], bupd_full[2], acc_full[2], tmem_empty[2], drain;
@@ -102,7 +105,7 @@ __device__ __forceinline__ int chan_of(int p) {
 __device__ __forceinline__ uint32_t sw128(int r, int chunk) { return (uint32_t)(r * 128 + ((chunk ^ (r & 7)) << 4)); }
 
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, const PoolDev& p, int* abort) {
-  if (mbar_wait_bounded(bar, parity, p.flags)) return true;
+  if (tc::mbar_wait_sleep(bar, parity, p.flags)) return true;
   *reinterpret_cast<volatile int*>(abort) = 1;
   return false;
 }
@@ -115,6 +118,13 @@ __device__ __forceinline__ int clampi(int x, int lo, int hi) { return x < lo ? l
 __device__ __forceinline__ int norm_exp(float m, int lim) {
   if (!(m >= 1.17549435e-38f) || !(m < INFINITY)) return 0;
   return clampi(14 - exp2_floor(m), -lim, lim);
+}
+
+// max of three that returns NaN if any input is NaN
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // First head index >= from (stepping by step, below end) due for a commit, or
@@ -175,11 +185,13 @@ __device__ void mma_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uint32_t 
   for (int k = 0;; ++k) {
     const int t = k & 1;
     if (!bounded_wait(&sm.tile_full[t], (uint32_t)((k >> 1) & 1), p, &sm.abort)) break;
-    if (sm.meta_head[t] < 0) {
+    // the epilogue has taken the head two back out of buffer t; this also
+    // keeps the end-of-work arrival below from running two phases ahead of it
+    if (k >= 2 && !bounded_wait(&sm.tmem_empty[t], (uint32_t)(((k - 2) >> 1) & 1), p, &sm.abort)) break;
+    if (sm.meta_head[k & 3] < 0) {
       tc::mbar_arrive(&sm.acc_full[t]);
       break;
     }
-    if (k >= 2 && !bounded_wait(&sm.tmem_empty[t], (uint32_t)(((k - 2) >> 1) & 1), p, &sm.abort)) break;
     tc::fence_after_sync();
     const uint32_t tile = smem_addr(sm.tile[t]), bx = smem_addr(sm.bx[t]);
     const uint32_t dC = tm + 256u * t, dU = dC + 128u;
@@ -208,27 +220,41 @@ __device__ void mma_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uint32_t 
   }
   // every product issued has completed before TMEM is released
   tc::commit(&sm.drain);
-  mbar_wait_bounded(&sm.drain, 0, p.flags);
+  tc::mbar_wait_sleep(&sm.drain, 0, p.flags);
 }
 
 // ---- converters --------------------------------------------------------------
 // Codes of one staged record -> the f16 tile (exact values), [jh][i][64
 // positions] with 128-byte swizzling.  Each lane converts 16 channels of one
 // row per step; a quarter-warp covers two rows whose halves are swapped, so
-// its loads and its 16-byte stores each fall in distinct banks.
+// its loads and its 16-byte stores each fall in distinct banks.  The eight
+// steps of a lane differ by constant offsets (the swizzle term depends only
+// on the row modulo 8, which is fixed per lane).
 template <int BITS>
 __device__ __forceinline__ void convert_codes(const uint8_t* rec, uint8_t* tile, int cw, int lane) {
   const uint32_t K64 = 0x64646464u;
-  const __half2 off8 = __float2half2_rn(1032.f), off16 = __float2half2_rn(72.f);
+  const __half2 off8 = __float2half2_rn(1032.f), off16 = __float2half2_rn(-72.f);
   const __half2 sixteenth = __float2half2_rn(0.0625f), off128 = __float2half2_rn(1152.f);
   const int qq = lane >> 3, r = (lane >> 2) & 1, mm = lane & 3;
-#pragma unroll 2
+  const int i0 = 32 * cw + 2 * qq + r;               // row of step 0; step it adds 8 (it >> 1)
+  const int r7 = i0 & 7;
+  // group of the even steps (m16 = 4 r + mm) and of the odd ones (m16 = 4 (1 - r) + mm)
+  const int mA = 4 * r + mm, mB = 4 * (1 - r) + mm;
+  const uint8_t* srcA = rec + (BITS == 4 ? 64 * i0 + 8 * mA : 128 * i0 + 16 * mA);
+  const uint8_t* srcB = rec + (BITS == 4 ? 64 * i0 + 8 * mB : 128 * i0 + 16 * mB);
+  uint8_t* dstA = tile + (mA >> 2) * 16384 + 128 * i0;
+  uint8_t* dstB = tile + (mB >> 2) * 16384 + 128 * i0;
+  const int cA0 = ((2 * (mA & 3)) ^ r7) << 4, cA1 = ((2 * (mA & 3) + 1) ^ r7) << 4;
+  const int cB0 = ((2 * (mB & 3)) ^ r7) << 4, cB1 = ((2 * (mB & 3) + 1) ^ r7) << 4;
+  const int rstride = BITS == 4 ? 512 : 1024;         // 8 rows of codes
+#pragma unroll
   for (int it = 0; it < 8; ++it) {
-    const int i = 32 * cw + 8 * (it >> 1) + 2 * qq + r;
-    const int m16 = 4 * ((it & 1) ^ r) + mm;          // 16-channel group
+    const bool odd = it & 1;
+    const uint8_t* src = (odd ? srcB : srcA) + rstride * (it >> 1);
+    uint8_t* dst = (odd ? dstB : dstA) + 1024 * (it >> 1);
     uint32_t hv[8];                                    // positions 16 m16 + 0..15 as f16 pairs
     if (BITS == 4) {
-      const uint2 w = *reinterpret_cast<const uint2*>(rec + 64 * i + 8 * m16);
+      const uint2 w = *reinterpret_cast<const uint2*>(src);
       // offset codes u = c + 8: even channels in the low nibbles, odd ones (x16) in the high
       const uint32_t x0 = (w.x & 0x0F0F0F0Fu) ^ 0x08080808u, y0 = (w.x & 0xF0F0F0F0u) ^ 0x80808080u;
       const uint32_t x1 = (w.y & 0x0F0F0F0Fu) ^ 0x08080808u, y1 = (w.y & 0xF0F0F0F0u) ^ 0x80808080u;
@@ -236,12 +262,12 @@ __device__ __forceinline__ void convert_codes(const uint8_t* rec, uint8_t* tile,
       hv[1] = h2u(__hsub2(u2h(prmt(x0, K64, 0x4342u)), off8));    // 4, 6
       hv[2] = h2u(__hsub2(u2h(prmt(x1, K64, 0x4140u)), off8));    // 8, 10
       hv[3] = h2u(__hsub2(u2h(prmt(x1, K64, 0x4342u)), off8));    // 12, 14
-      hv[4] = h2u(__hfma2(u2h(prmt(y0, K64, 0x4140u)), sixteenth, __hneg2(off16)));   // 1, 3
-      hv[5] = h2u(__hfma2(u2h(prmt(y0, K64, 0x4342u)), sixteenth, __hneg2(off16)));   // 5, 7
-      hv[6] = h2u(__hfma2(u2h(prmt(y1, K64, 0x4140u)), sixteenth, __hneg2(off16)));   // 9, 11
-      hv[7] = h2u(__hfma2(u2h(prmt(y1, K64, 0x4342u)), sixteenth, __hneg2(off16)));   // 13, 15
+      hv[4] = h2u(__hfma2(u2h(prmt(y0, K64, 0x4140u)), sixteenth, off16));   // 1, 3
+      hv[5] = h2u(__hfma2(u2h(prmt(y0, K64, 0x4342u)), sixteenth, off16));   // 5, 7
+      hv[6] = h2u(__hfma2(u2h(prmt(y1, K64, 0x4140u)), sixteenth, off16));   // 9, 11
+      hv[7] = h2u(__hfma2(u2h(prmt(y1, K64, 0x4342u)), sixteenth, off16));   // 13, 15
     } else {
-      const uint4 w = *reinterpret_cast<const uint4*>(rec + 128 * i + 16 * m16);
+      const uint4 w = *reinterpret_cast<const uint4*>(src);
       const uint32_t ws[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u, w.z ^ 0x80808080u, w.w ^ 0x80808080u};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -249,10 +275,8 @@ __device__ __forceinline__ void convert_codes(const uint8_t* rec, uint8_t* tile,
         hv[2 * e + 1] = h2u(__hsub2(u2h(prmt(ws[e], K64, 0x4342u)), off128));
       }
     }
-    uint8_t* base = tile + (m16 >> 2) * 16384;
-    const int ch = 2 * (m16 & 3);
-    *reinterpret_cast<uint4*>(base + sw128(i, ch)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    *reinterpret_cast<uint4*>(base + sw128(i, ch + 1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+    *reinterpret_cast<uint4*>(dst + (odd ? cB0 : cA0)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<uint4*>(dst + (odd ? cB1 : cA1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
   }
 }
 
@@ -268,114 +292,134 @@ __device__ __forceinline__ KeyExp key_exponents(const float* G, int P) {
 // The scaled keys of one head: B of X (rows s: hi, PMAX + s: lo of
 // s_j k_s[j] 2^exx) and A of the update (rows s and PMAX + s: k_s[j] 2^exk
 // in f16, and rows 2 PMAX + s: its low part for fp32 rows), by tile
-// position.  Tokens s >= n give zero rows.
+// position.  Thread ct owns the position pair 2 (ct % 64) + {0, 1} and half
+// of the tokens.  Tokens s >= n give zero rows.
 template <bool BF16, bool R8, int PMAX, int BITS>
 __device__ __forceinline__ void build_keys(const uint8_t* stage, uint8_t* bx, uint8_t* au, int n, KeyExp ex, int ct) {
   using C = TcCfg<BF16, R8, PMAX>;
   const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + code_bytes(C::D, C::D, BITS));
   const uint8_t* rows = stage + C::REC;
+  const int pp = ct & 63, s0 = (ct >> 6) * (PMAX / 2);
+  const int j0 = chan_of<BITS>(2 * pp), j1 = chan_of<BITS>(2 * pp + 1);
   const float upx = pow2i(ex.exx), upk = pow2i(ex.exk);
-  for (int u = ct; u < PMAX * 16; u += 128) {
-    const int s = u >> 4, c16 = u & 15;                // token, 8-position chunk
-    uint32_t bh[4], bl[4], kh[4], kl[4];
+  const float2 sx = make_float2(__half2float(__ushort_as_half(sc[j0])) * upx,
+                                __half2float(__ushort_as_half(sc[j1])) * upx);
+  const float2 uk = make_float2(upk, upk);
+  // byte offset of the pair inside a [rows][64] 128B-swizzled block: chunk (pp % 32) / 4, word pp % 4
+  const int half = pp >> 5, chunk = (pp & 31) >> 2, word = (pp & 3) * 4;
+  uint8_t* xb = bx + half * (C::NX * 128) + word;
+  uint8_t* ab = au + half * (C::KU * 128) + word;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float b2[2], k2[2];
-#pragma unroll
-      for (int z = 0; z < 2; ++z) {
-        const int j = chan_of<BITS>(8 * c16 + 2 * e + z);
-        const float kv = s < n ? row_at<R8>(rows + s * C::ROWB, j, BF16) : 0.f;
-        b2[z] = s < n ? kv * __half2float(__ushort_as_half(sc[j])) * upx : 0.f;
-        k2[z] = kv * upk;
-      }
-      const __half2 bhi = __floats2half2_rn(b2[0], b2[1]);
-      const float2 bhf = __half22float2(bhi);
-      bh[e] = h2u(bhi);
-      bl[e] = h2u(__floats2half2_rn(b2[0] - bhf.x, b2[1] - bhf.y));
-      const __half2 khi = __floats2half2_rn(k2[0], k2[1]);
-      const float2 khf = __half22float2(khi);
-      kh[e] = h2u(khi);
-      kl[e] = h2u(__floats2half2_rn(k2[0] - khf.x, k2[1] - khf.y));
+  for (int s = s0; s < s0 + PMAX / 2; ++s) {
+    float2 kv = make_float2(0.f, 0.f);
+    if (s < n) {
+      kv.x = row_at<R8>(rows + s * C::ROWB, j0, BF16);
+      kv.y = row_at<R8>(rows + s * C::ROWB, j1, BF16);
     }
-    uint8_t* xb = bx + (c16 >> 3) * (C::NX * 128);
-    const int ch = c16 & 7;
-    *reinterpret_cast<uint4*>(xb + sw128(s, ch)) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
-    *reinterpret_cast<uint4*>(xb + sw128(PMAX + s, ch)) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
-    uint8_t* ab = au + (c16 >> 3) * (C::KU * 128);
-    *reinterpret_cast<uint4*>(ab + sw128(s, ch)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-    *reinterpret_cast<uint4*>(ab + sw128(PMAX + s, ch)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-    if (C::NSEG == 3)
-      *reinterpret_cast<uint4*>(ab + sw128(2 * PMAX + s, ch)) = make_uint4(kl[0], kl[1], kl[2], kl[3]);
+    const float2 b = __fmul2_rn(kv, sx);
+    const __half2 bh = __float22half2_rn(b);
+    const float2 bhf = __half22float2(bh);
+    const __half2 bl = __float22half2_rn(make_float2(b.x - bhf.x, b.y - bhf.y));
+    const float2 k2 = __fmul2_rn(kv, uk);
+    const __half2 kh = __float22half2_rn(k2);
+    *reinterpret_cast<uint32_t*>(xb + sw128(s, chunk)) = h2u(bh);
+    *reinterpret_cast<uint32_t*>(xb + sw128(PMAX + s, chunk)) = h2u(bl);
+    *reinterpret_cast<uint32_t*>(ab + sw128(s, chunk)) = h2u(kh);
+    *reinterpret_cast<uint32_t*>(ab + sw128(PMAX + s, chunk)) = h2u(kh);
+    if (C::NSEG == 3) {
+      const float2 khf = __half22float2(kh);
+      *reinterpret_cast<uint32_t*>(ab + sw128(2 * PMAX + s, chunk)) =
+          h2u(__float22half2_rn(make_float2(k2.x - khf.x, k2.y - khf.y)));
+    }
   }
 }
 
 // R and U^ for one head, one TMEM lane (value channel i) per converter thread:
 // x_s from TMEM, r_s = v_s[i] - gamma_s x_s, U^[s][i] = sum_s' W[s][s'] r_s',
 // normalised by one power of two for the head, split hi + lo into row i of
-// the update's B.  Also the epilogue's per-position factors.
-template <bool BF16, bool R8, int PMAX, int BITS>
+// the update's B.  Also the epilogue's per-position factors.  A head with
+// all PMAX tokens takes packed pair arithmetic over the factor rows; early
+// commits (n < PMAX) take guarded scalar loops.
+template <bool BF16, bool R8, int PMAX>
 __device__ __forceinline__ void residual_update(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, const uint8_t* stage,
-                                                int t, int n, uint32_t tm, int k, int ct, int warp, int lane) {
+                                                int bits, int t, int n, uint32_t tm, int k, int ct, int warp,
+                                                int lane) {
   using C = TcCfg<BF16, R8, PMAX>;
+  const int m = k & 3;   // ring slot of this head
   const int P = p.P;
   const int qd = warp & 3, i = 32 * qd + lane;
-  uint32_t xr[2 * PMAX];
-  {
-    uint32_t tmp[16];
-    tc::ld_32x32b_x16(tm + ((uint32_t)(32 * qd) << 16) + 256u * t + 128u, tmp);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) xr[c] = tmp[c];
-    if (PMAX == 16) {
-      tc::ld_32x32b_x16(tm + ((uint32_t)(32 * qd) << 16) + 256u * t + 144u, tmp);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) xr[(16 + c) % (2 * PMAX)] = tmp[c];
-    }
-    tc::wait_ld();
-  }
   const float* G = reinterpret_cast<const float*>(stage + C::REC + C::KVB);
   const float* W = G;
   const float* gam = G + P * P;
   const KeyExp ex = key_exponents(G, P);
   const float xinv = pow2i(-ex.exx);
-  const uint8_t* rows = stage + C::REC;
-  float r[PMAX];
+  const uint8_t* vrow = stage + C::REC + C::D * C::ESZ + i * C::ESZ;   // v_0[i]
+  float x[PMAX], r[PMAX], u[PMAX];
+  {
+    uint32_t xa[16], xb[16];
+    tc::ld_32x32b_x16(tm + ((uint32_t)(32 * qd) << 16) + 256u * t + 128u, xa);
+    if (PMAX == 16) tc::ld_32x32b_x16(tm + ((uint32_t)(32 * qd) << 16) + 256u * t + 144u, xb);
+    tc::wait_ld();
 #pragma unroll
-  for (int s = 0; s < PMAX; ++s) {
-    const float x = (__uint_as_float(xr[s]) + __uint_as_float(xr[PMAX + s])) * xinv;
-    r[s] = s < n ? row_at<R8>(rows + s * C::ROWB, C::D + i, BF16) - gam[s] * x : 0.f;
-  }
-  float u[PMAX];
-  float um = 0.f;
-#pragma unroll
-  for (int s = 0; s < PMAX; ++s) {
-    float a = 0.f;
-    if (s < n) {
-      if ((P & 3) == 0) {
-#pragma unroll
-        for (int c = 0; c < PMAX / 4; ++c) {
-          if (4 * c < P) {
-            const float4 w4 = *reinterpret_cast<const float4*>(W + s * P + 4 * c);
-            a = fmaf(w4.x, r[4 * c], a);
-            a = fmaf(w4.y, r[4 * c + 1], a);
-            a = fmaf(w4.z, r[4 * c + 2], a);
-            a = fmaf(w4.w, r[4 * c + 3], a);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int sp = 0; sp < PMAX; ++sp)
-          if (sp < n) a = fmaf(W[s * P + sp], r[sp], a);
-      }
+    for (int s2 = 0; s2 < PMAX; s2 += 2) {
+      const int h0 = s2, l0 = PMAX + s2;   // hi and lo columns of tokens s2, s2 + 1
+      const float2 hi = make_float2(__uint_as_float(h0 < 16 ? xa[h0] : xb[h0 - 16]),
+                                    __uint_as_float(h0 + 1 < 16 ? xa[h0 + 1] : xb[h0 - 15]));
+      const float2 lo = make_float2(__uint_as_float(l0 < 16 ? xa[l0] : xb[l0 - 16]),
+                                    __uint_as_float(l0 + 1 < 16 ? xa[l0 + 1] : xb[l0 - 15]));
+      const float2 xs = __fadd2_rn(hi, lo);
+      x[s2] = xs.x;
+      x[s2 + 1] = xs.y;
     }
-    u[s] = a;
-    um = max_nan(um, fabsf(a));
+  }
+  const bool full = n == PMAX && P == PMAX;
+  float um;
+  if (full) {
+#pragma unroll
+    for (int s2 = 0; s2 < PMAX; s2 += 2) {
+      const float2 g = __fmul2_rn(*reinterpret_cast<const float2*>(gam + s2), make_float2(-xinv, -xinv));
+      const float2 v = make_float2(row_at<R8>(vrow + s2 * C::ROWB, 0, BF16), row_at<R8>(vrow + (s2 + 1) * C::ROWB, 0, BF16));
+      const float2 rr = __ffma2_rn(g, make_float2(x[s2], x[s2 + 1]), v);
+      r[s2] = rr.x;
+      r[s2 + 1] = rr.y;
+    }
+    float2 mu = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < PMAX; ++s) {
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < PMAX; c += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(W + s * PMAX + c);
+        acc = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(r[c], r[c + 1]), acc);
+        acc = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(r[c + 2], r[c + 3]), acc);
+      }
+      u[s] = acc.x + acc.y;
+    }
+    um = 0.f;
+#pragma unroll
+    for (int s = 0; s < PMAX; s += 2) um = max3_nan(um, fabsf(u[s]), fabsf(u[s + 1]));
+    (void)mu;
+  } else {
+#pragma unroll
+    for (int s = 0; s < PMAX; ++s)
+      r[s] = s < n ? row_at<R8>(vrow + s * C::ROWB, 0, BF16) - gam[s] * (x[s] * xinv) : 0.f;
+    um = 0.f;
+#pragma unroll
+    for (int s = 0; s < PMAX; ++s) {
+      float a = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < PMAX; ++sp)
+        if (s < n && sp < n) a = fmaf(W[s * P + sp], r[sp], a);
+      u[s] = a;
+      um = max_nan(um, fabsf(a));
+    }
   }
   // one exponent for the head's U^ (all 128 lanes feed one product)
 #pragma unroll
   for (int off = 16; off; off >>= 1) um = max_nan(um, __shfl_xor_sync(FULL, um, off));
   if (lane == 0) sm.red[k & 1][warp - C::CONV0] = um;
   tc::named_sync(6, 128);
-  um = max_nan(max_nan(sm.red[k & 1][0], sm.red[k & 1][1]), max_nan(sm.red[k & 1][2], sm.red[k & 1][3]));
+  um = max3_nan(max_nan(sm.red[k & 1][0], sm.red[k & 1][1]), sm.red[k & 1][2], sm.red[k & 1][3]);
   int e_tot = ex.exk + norm_exp(um, 40);
   const float smax = G[P * P + P + 1];
   if (smax >= 1.17549435e-38f && smax < INFINITY) e_tot = min(e_tot, 111 - exp2_floor(smax));
@@ -384,27 +428,26 @@ __device__ __forceinline__ void residual_update(const PoolDev& p, TcSmem<BF16, R
   uint32_t hi[PMAX / 2], lo[PMAX / 2];
 #pragma unroll
   for (int e = 0; e < PMAX / 2; ++e) {
-    const float a = u[2 * e] * up, b = u[2 * e + 1] * up;
-    const __half2 h = __floats2half2_rn(a, b);
+    const float2 a = __fmul2_rn(make_float2(u[2 * e], u[2 * e + 1]), make_float2(up, up));
+    const __half2 h = __float22half2_rn(a);
     const float2 hf = __half22float2(h);
     hi[e] = h2u(h);
-    lo[e] = h2u(__floats2half2_rn(a - hf.x, b - hf.y));
+    lo[e] = h2u(__float22half2_rn(make_float2(a.x - hf.x, a.y - hf.y)));
   }
   uint8_t* row = sm.bu[t] + (i >> 3) * 256 + (i & 7) * 16;
-  auto put = [&](int kk0, const uint32_t* src) {   // 8 K entries starting at kk0 (a multiple of 8)
-    *reinterpret_cast<uint4*>(row + (kk0 >> 4) * 4096 + ((kk0 >> 3) & 1) * 128) =
-        make_uint4(src[0], src[1], src[2], src[3]);
-  };
 #pragma unroll
   for (int c = 0; c < PMAX / 8; ++c) {
-    put(8 * c, hi + 4 * c);
-    put(PMAX + 8 * c, lo + 4 * c);
-    if (C::NSEG == 3) put(2 * PMAX + 8 * c, hi + 4 * c);
+    const int k0 = 8 * c, k1 = PMAX + 8 * c, k2 = 2 * PMAX + 8 * c;
+    *reinterpret_cast<uint4*>(row + (k0 >> 4) * 4096 + ((k0 >> 3) & 1) * 128) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+    *reinterpret_cast<uint4*>(row + (k1 >> 4) * 4096 + ((k1 >> 3) & 1) * 128) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+    if (C::NSEG == 3)
+      *reinterpret_cast<uint4*>(row + (k2 >> 4) * 4096 + ((k2 >> 3) & 1) * 128) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
   }
   // epilogue factors, one tile position per thread
-  const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + code_bytes(C::D, C::D, BITS));
-  sm.fj[t][ct] = gam[n - 1] * __half2float(__ushort_as_half(sc[chan_of<BITS>(ct)])) * pow2i(e_tot);
-  if (ct == 0) sm.meta_e[t] = e_tot;
+  const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + code_bytes(C::D, C::D, bits));
+  const int j = bits == 4 ? chan_of<4>(ct) : ct;
+  sm.fj[m][ct] = gam[n - 1] * __half2float(__ushort_as_half(sc[j])) * pow2i(e_tot);
+  if (ct == 0) sm.meta_e[m] = e_tot;
 }
 
 template <bool BF16, bool R8, int PMAX>
@@ -414,31 +457,32 @@ __device__ void converter_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uin
   // Every wait is followed by a vote at the converters' named barrier, so that
   // the four warps leave together and none is left waiting in a barrier.
   for (int k = 0;; ++k) {
-    const int s = k % C::NST, t = k & 1;
+    const int s = k % C::NST, t = k & 1, m = k & 3;
     bool ok = bounded_wait(&sm.stage_full[s], (uint32_t)((k / C::NST) & 1), p, &sm.abort);
     const int head = ok ? sm.stage_head[s] : -1;
-    // buffer t is free once the epilogue of the head two back has read its
-    // metadata and factors and released its TMEM (its update, which read this
-    // buffer's keys, is then done as well)
-    if (ok && k >= 2) ok = bounded_wait(&sm.tmem_empty[t], (uint32_t)(((k - 2) >> 1) & 1), p, &sm.abort);
+    if (tc::named_sync_any(6, 128, !ok)) return;
+    const uint8_t* st = sm.stage[s];
+    const int bits = head >= 0 ? p.bits[head % p.H] : 4;
+    // the tile and X's keys of buffer t were last read by the products of the
+    // head two back, whose completion the previous R step waited for
+    if (head >= 0) {
+      if (bits == 4) convert_codes<4>(st, sm.tile[t], cw, lane);
+      else convert_codes<8>(st, sm.tile[t], cw, lane);
+    }
+    // the update of the head two back read this buffer's update keys; its
+    // completion also means the epilogue of the head four back, which used
+    // this ring slot, has read it
+    if (k >= 2) ok = bounded_wait(&sm.acc_full[t], (uint32_t)(((k - 2) >> 1) & 1), p, &sm.abort);
     if (tc::named_sync_any(6, 128, !ok)) return;
     if (head >= 0) {
-      const uint8_t* st = sm.stage[s];
       const int n = sm.stage_n[s];
       const KeyExp ex = key_exponents(reinterpret_cast<const float*>(st + C::REC + C::KVB), p.P);
-      if (p.bits[head % p.H] == 4) {
-        convert_codes<4>(st, sm.tile[t], cw, lane);
-        build_keys<BF16, R8, PMAX, 4>(st, sm.bx[t], sm.au[t], n, ex, ct);
-      } else {
-        convert_codes<8>(st, sm.tile[t], cw, lane);
-        build_keys<BF16, R8, PMAX, 8>(st, sm.bx[t], sm.au[t], n, ex, ct);
-      }
-      if (ct == 0) {
-        sm.meta_head[t] = head;
-        sm.meta_n[t] = n;
-      }
-    } else if (ct == 0) {
-      sm.meta_head[t] = -1;
+      if (bits == 4) build_keys<BF16, R8, PMAX, 4>(st, sm.bx[t], sm.au[t], n, ex, ct);
+      else build_keys<BF16, R8, PMAX, 8>(st, sm.bx[t], sm.au[t], n, ex, ct);
+    }
+    if (ct == 0) {
+      sm.meta_head[m] = head;
+      sm.meta_bits[m] = bits;
     }
     fence_proxy_async_smem();
     tc::mbar_arrive(&sm.tile_full[t]);
@@ -448,10 +492,8 @@ __device__ void converter_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uin
       if (tc::named_sync_any(6, 128, !ok)) return;
       tc::fence_after_sync();
       const int hp = sm.stage_head[sp];
-      if (p.bits[hp % p.H] == 4)
-        residual_update<BF16, R8, PMAX, 4>(p, sm, sm.stage[sp], tp, sm.stage_n[sp], tm, k - 1, ct, warp, lane);
-      else
-        residual_update<BF16, R8, PMAX, 8>(p, sm, sm.stage[sp], tp, sm.stage_n[sp], tm, k - 1, ct, warp, lane);
+      residual_update<BF16, R8, PMAX>(p, sm, sm.stage[sp], p.bits[hp % p.H], tp, sm.stage_n[sp], tm, k - 1, ct,
+                                      warp, lane);
       fence_proxy_async_smem();
       tc::fence_before_sync();
       tc::mbar_arrive(&sm.bupd_full[tp]);
@@ -462,66 +504,81 @@ __device__ void converter_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uin
 }
 
 // ---- epilogue ----------------------------------------------------------------
-// Thread (g = lane / 4, q = lane % 4) of warp we holds, for 16-lane blocks blk
-// of its quadrant qd, tile positions p = 32 qd + 16 blk + g + 8 h (h = 0, 1)
-// and value channels i = 64 hf + 8 c + 2 q + {0, 1} (c = 0..7): 64 elements
-// of S'^T = S^T 2^e.  INT4 tile positions pair the key channels 2m (h = 0)
-// and 2m + 1 (h = 1) in one thread, so a code byte is thread-local.
+// Four warps, one per TMEM lane quadrant qd.  Thread (g = lane / 4, q = lane % 4)
+// holds, for 16-lane blocks blk of the quadrant, tile positions p = 32 qd +
+// 16 blk + g + 8 h (h = 0, 1) and value channels i = 64 cb + 8 c + 2 q + {0, 1}
+// (column half cb = 0, 1; c = 0..7): 128 elements of S'^T = S^T 2^e, four key
+// channels of 32 values each.  INT4 tile positions pair the key channels 2m
+// (h = 0) and 2m + 1 (h = 1) in one thread, so a code byte is thread-local.
+
+// Codes of two values as the low byte (INT8) or low nibble (INT4) of each
+// f16 half: x q + 1280 (resp. 1040) rounded to f16 is the integer 1280 + c
+// (1040 + c) with c = rint_half_even(x q), whose mantissa's low byte is c
+// modulo 256 (low nibble c modulo 16).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_pair_fast(float a, float b, float q) {
+  const float M = BITS == 4 ? 1040.f : 1280.f;
+  return h2u(__float22half2_rn(__ffma2_rn(make_float2(a, b), make_float2(q, q), make_float2(M, M))));
+}
+// Same layout from the exact encoder (fp32 divide by the scale).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_pair_exact(float a, float b, float sf) {
+  const int qmax = BITS == 4 ? 7 : 127, off = BITS == 4 ? 16 : 256;
+  const uint32_t ca = (uint32_t)(encode_value(a, sf, qmax) + off), cb = (uint32_t)(encode_value(b, sf, qmax) + off);
+  return (0x6400u + ca) | ((0x6400u + cb) << 16);
+}
+
 template <bool BF16, bool R8, int PMAX, int BITS>
 __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps& maps, TcSmem<BF16, R8, PMAX>& sm,
-                                              uint32_t tm, int t, int head, int we, int lane) {
+                                              uint32_t tm, int t, int m, int head, int we, int lane) {
   using C = TcCfg<BF16, R8, PMAX>;
-  const int qd = we & 3, hf = (we - C::EPI0) >> 2, g = lane >> 2, q = lane & 3;
-  const int e_tot = sm.meta_e[t];
+  const int qd = we & 3, g = lane >> 2, q = lane & 3;
+  const int e_tot = sm.meta_e[m];
   const float down = pow2i(-e_tot);
-  float S[2][32];
-  {
-    float f[2][2];
+  float f[2][2];
 #pragma unroll
-    for (int blk = 0; blk < 2; ++blk)
+  for (int blk = 0; blk < 2; ++blk)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) f[blk][h] = sm.fj[t][32 * qd + 16 * blk + g + 8 * h];
+    for (int h = 0; h < 2; ++h) f[blk][h] = sm.fj[m][32 * qd + 16 * blk + g + 8 * h];
+  // S'^T of block blk, column half cb: v[4 c + 2 h + z] = rows 64 cb + 8 c + 2 q + z of lane g + 8 h
+  auto load = [&](int blk, int cb, float (&v)[32]) {
+    uint32_t cr[32], ur[32];
+    const uint32_t a = tm + ((uint32_t)(32 * qd + 16 * blk) << 16) + 256u * t + 64u * cb;
+    tc::ld_16x256b_x8(a, cr);
+    tc::ld_16x256b_x8(a + 128u, ur);
+    tc::wait_ld();
 #pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-      uint32_t cr[32], ur[32];
-      const uint32_t lb = (uint32_t)(32 * qd + 16 * blk) << 16;
-      tc::ld_16x256b_x8(tm + lb + 256u * t + 64u * hf, cr);
-      tc::ld_16x256b_x8(tm + lb + 256u * t + 128u + 64u * hf, ur);
-      tc::wait_ld();
+    for (int c = 0; c < 8; ++c)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 r2 = __ffma2_rn(make_float2(__uint_as_float(cr[4 * c + 2 * h]), __uint_as_float(cr[4 * c + 2 * h + 1])),
+                                     make_float2(f[blk][h], f[blk][h]),
+                                     make_float2(__uint_as_float(ur[4 * c + 2 * h]), __uint_as_float(ur[4 * c + 2 * h + 1])));
+        v[4 * c + 2 * h] = r2.x;
+        v[4 * c + 2 * h + 1] = r2.y;
+      }
+  };
+
+  // pass 1: column maxima, 32 values per key channel here, then the other three lanes of the quad
+  float mx[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+      float v[32];
+      load(blk, cb, v);
 #pragma unroll
       for (int c = 0; c < 8; ++c)
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          S[blk][4 * c + k] = fmaf(__uint_as_float(cr[4 * c + k]), f[blk][k >> 1], __uint_as_float(ur[4 * c + k]));
+        for (int h = 0; h < 2; ++h) mx[blk][h] = max3_nan(mx[blk][h], fabsf(v[4 * c + 2 * h]), fabsf(v[4 * c + 2 * h + 1]));
     }
-  }
-  tc::fence_before_sync();
-  tc::mbar_arrive(&sm.tmem_empty[t]);
-
-  // column maxima: 16 values per (blk, h) here, the other three lanes of the
-  // quad, then the warp holding the other 64 value channels
-  float m[2][2];
 #pragma unroll
   for (int blk = 0; blk < 2; ++blk)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float a = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) a = max_nan(a, max_nan(fabsf(S[blk][4 * c + 2 * h]), fabsf(S[blk][4 * c + 2 * h + 1])));
-      a = max_nan(a, __shfl_xor_sync(FULL, a, 1));
-      a = max_nan(a, __shfl_xor_sync(FULL, a, 2));
-      m[blk][h] = a;
+      mx[blk][h] = max_nan(mx[blk][h], __shfl_xor_sync(FULL, mx[blk][h], 1));
+      mx[blk][h] = max_nan(mx[blk][h], __shfl_xor_sync(FULL, mx[blk][h], 2));
     }
-  if (q == 0)
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) sm.amax_x[hf][32 * qd + 16 * blk + g + 8 * h] = m[blk][h];
-  tc::named_sync(1 + qd, 64);
-#pragma unroll
-  for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) m[blk][h] = max_nan(m[blk][h], sm.amax_x[hf ^ 1][32 * qd + 16 * blk + g + 8 * h]);
 
   // scale of the column (blk, h) = (q >> 1, q & 1), then shared across the quad
   const int qmax = BITS == 4 ? 7 : 127;
@@ -530,51 +587,71 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
   bool bad;
   {
     const int pos = 32 * qd + 16 * (q >> 1) + g + 8 * (q & 1);
-    const float amax = m[q >> 1][q & 1] * down;
-    const GroupScale gs = group_scale(amax, isfinite(amax), qmax, hf == 0 ? p.flags : nullptr);
+    const float amax = mx[q >> 1][q & 1] * down;
+    const GroupScale gs = group_scale(amax, isfinite(amax), qmax, p.flags);
     sf = gs.sf;
     qf = gs.sf > 0.f ? __frcp_rn(gs.sf) * down : 0.f;
     bad = !isfinite(amax) || (gs.bits == 0x7BFF && amax / qmax > 65504.f) || !(qf < INFINITY);
-    if (hf == 0) reinterpret_cast<uint16_t*>(stg + 16384)[chan_of<BITS>(pos)] = gs.bits;
-  }
-  float qv[2][2], sv[2][2];
-#pragma unroll
-  for (int z = 0; z < 4; ++z) {
-    qv[z >> 1][z & 1] = __shfl_sync(FULL, qf, (lane & ~3) | z);
-    sv[z >> 1][z & 1] = __shfl_sync(FULL, sf, (lane & ~3) | z);
+    reinterpret_cast<uint16_t*>(stg + 16384)[chan_of<BITS>(pos)] = gs.bits;
   }
   const bool slow = __any_sync(FULL, bad);
+  float qv[2][2];
+#pragma unroll
+  for (int z = 0; z < 4; ++z) qv[z >> 1][z & 1] = __shfl_sync(FULL, slow ? sf : qf, (lane & ~3) | z);
 
-  // codes: f16 magic pairs (rows 2q, 2q + 1 of one column), bytes gathered and
-  // stored transposed into the swizzled staging rows
-  auto pair = [&](int blk, int c, int h) -> uint32_t {
-    const float a = S[blk][4 * c + 2 * h], b = S[blk][4 * c + 2 * h + 1];
-    if (!slow) return magic_fast<BITS>(a, b, qv[blk][h], qv[blk][h]);
-    return magic_exact<BITS>(a * down, b * down, sv[blk][h], sv[blk][h]);
-  };
+  // pass 2: codes, gathered and stored transposed (four 8-row matrices per
+  // stmatrix) into the swizzled staging rows; lane l gives the address of
+  // row l % 8 of matrix l / 8
   const uint32_t stg_a = smem_addr(stg);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const int i = 64 * hf + 8 * c + (lane & 7);     // the staging row whose address this lane gives
+  const int r8 = lane & 7, mq = lane >> 3;
+  auto encode = [&](auto fast) {
+    auto pair = [&](const float (&v)[32], int blk, int c, int h) -> uint32_t {
+      if (decltype(fast)::value) return code_pair_fast<BITS>(v[4 * c + 2 * h], v[4 * c + 2 * h + 1], qv[blk][h]);
+      return code_pair_exact<BITS>(v[4 * c + 2 * h] * down, v[4 * c + 2 * h + 1] * down, qv[blk][h]);
+    };
     if (BITS == 4) {
-      uint32_t rb[2];
+      const uint32_t base = stg_a + 64 * r8 + ((qd ^ ((r8 >> 1) & 3)) << 4) + 512 * mq;
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        const uint32_t ev = pair(blk, c, 0), od = pair(blk, c, 1);
-        rb[blk] = ev | ((od << 4) & 0x00F000F0u);
+      for (int cb = 0; cb < 2; ++cb) {
+        uint32_t rb[2][8];   // [blk][c]: bytes 0 and 2 are the row pairs' code bytes
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          float v[32];
+          load(blk, cb, v);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            rb[blk][c] = (pair(v, blk, c, 0) & 0x000F000Fu) | ((pair(v, blk, c, 1) << 4) & ~0x000F000Fu);
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < 8; c0 += 4)
+          tc::stsm_trans_b8_x4(base + 512u * (8 * cb + c0), prmt(rb[0][c0], rb[1][c0], 0x6420u),
+                               prmt(rb[0][c0 + 1], rb[1][c0 + 1], 0x6420u), prmt(rb[0][c0 + 2], rb[1][c0 + 2], 0x6420u),
+                               prmt(rb[0][c0 + 3], rb[1][c0 + 3], 0x6420u));
       }
-      const uint32_t v = prmt(rb[0], rb[1], 0x6420u) ^ 0x88888888u;
-      tc::stsm_trans_b8(stg_a + 64 * i + ((qd ^ ((i >> 1) & 3)) << 4), v);
     } else {
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
-        const uint32_t v = prmt(pair(blk, c, 0), pair(blk, c, 1), 0x6420u) ^ 0x80808080u;
-        tc::stsm_trans_b8(stg_a + 128 * i + (((2 * qd + blk) ^ (i & 7)) << 4), v);
+        const uint32_t base = stg_a + 128 * r8 + (((2 * qd + blk) ^ r8) << 4) + 1024 * mq;
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+          float v[32];
+          load(blk, cb, v);
+          uint32_t w[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) w[c] = prmt(pair(v, blk, c, 0), pair(v, blk, c, 1), 0x6420u);
+#pragma unroll
+          for (int c0 = 0; c0 < 8; c0 += 4)
+            tc::stsm_trans_b8_x4(base + 1024u * (8 * cb + c0), w[c0], w[c0 + 1], w[c0 + 2], w[c0 + 3]);
+        }
       }
     }
-  }
+  };
+  if (!slow) encode(std::true_type{});
+  else encode(std::false_type{});
+  tc::fence_before_sync();
+  tc::mbar_arrive(&sm.tmem_empty[t]);
   fence_proxy_async_smem();
-  tc::named_sync(5, 256);
+  tc::named_sync(5, 128);
   if (we == C::EPI0 && lane == 0) {
     const int hh = head % p.H, b = head / p.H;
     const size_t off = (size_t)b * p.slot_stride + p.rec_off[hh];
@@ -591,15 +668,17 @@ template <bool BF16, bool R8, int PMAX>
 __device__ void epilogue_role(const PoolDev& p, const CommitMaps& maps, TcSmem<BF16, R8, PMAX>& sm, uint32_t tm,
                               int warp, int lane) {
   for (int k = 0;; ++k) {
-    const int t = k & 1;
-    // the eight warps vote after the wait and leave together (named barriers follow)
-    const bool ok = bounded_wait(&sm.acc_full[t], (uint32_t)((k >> 1) & 1), p, &sm.abort);
-    if (tc::named_sync_any(5, 256, !ok)) break;
+    const int t = k & 1, m = k & 3;
+    // the four warps vote after the wait and leave together (named barriers follow)
+    bool ok = bounded_wait(&sm.acc_full[t], (uint32_t)((k >> 1) & 1), p, &sm.abort);
+    // the converters' per-head values (factors, exponent) are read directly after their arrival
+    if (ok && sm.meta_head[m] >= 0) ok = bounded_wait(&sm.bupd_full[t], (uint32_t)((k >> 1) & 1), p, &sm.abort);
+    if (tc::named_sync_any(5, 128, !ok)) break;
     tc::fence_after_sync();
-    const int head = sm.meta_head[t];
+    const int head = sm.meta_head[m];
     if (head < 0) break;
-    if (p.bits[head % p.H] == 4) epilogue_head<BF16, R8, PMAX, 4>(p, maps, sm, tm, t, head, warp, lane);
-    else epilogue_head<BF16, R8, PMAX, 8>(p, maps, sm, tm, t, head, warp, lane);
+    if (sm.meta_bits[m] == 4) epilogue_head<BF16, R8, PMAX, 4>(p, maps, sm, tm, t, m, head, warp, lane);
+    else epilogue_head<BF16, R8, PMAX, 8>(p, maps, sm, tm, t, m, head, warp, lane);
   }
   if (warp == TcCfg<BF16, R8, PMAX>::EPI0 && lane == 0) tc::bulk_wait_all();
 }
@@ -624,7 +703,7 @@ __global__ void __launch_bounds__(TcCfg<BF16, R8, PMAX>::THREADS, 1)
       mbar_init(&sm.x_full[t], 1);
       mbar_init(&sm.bupd_full[t], 128);
       mbar_init(&sm.acc_full[t], 1);
-      mbar_init(&sm.tmem_empty[t], 256);
+      mbar_init(&sm.tmem_empty[t], 128);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;

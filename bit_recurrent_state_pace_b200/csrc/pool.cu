@@ -13,6 +13,7 @@ struct pace_pool {
   // tensor maps of the state region for the tensor-memory commit (d = 128)
   pace::CommitMaps maps;
   bool maps_ok = false;
+  int32_t commit_engine = PACE_COMMIT_MMA;
   pace_pool_desc desc;
   size_t state_bytes, buffer_bytes, aux_bytes, kv_bytes;
   size_t rec_bytes[PACE_MAX_HEADS];
@@ -36,11 +37,11 @@ inline pace_status from_cuda(cudaError_t e) {
   return PACE_ERR_CUDA;
 }
 
-// Period commit of the heads due in a span: the tensor-memory kernel for the
-// shapes it is built for, the mma.sync kernel otherwise.
+// Period commit of the heads due in a span, by the pool's commit engine.
 inline cudaError_t commit_launch(const pace_pool* pool, const pace::PoolDev& dev, const pace::Span& sp,
                                  cudaStream_t st) {
-  if (pool->maps_ok && pace::commit_tc_supported(dev)) return pace::launch_commit_tc(dev, sp, pool->maps, st);
+  if (pool->commit_engine == PACE_COMMIT_TCGEN05 && pool->maps_ok && pace::commit_tc_supported(dev))
+    return pace::launch_commit_tc(dev, sp, pool->maps, st);
   return pace::launch_commit(dev, sp, st);
 }
 
@@ -250,6 +251,14 @@ pace_status pace_set_commit_threshold(pace_pool* pool, float tau) {
   if (pool->dev.row8 && std::isfinite(tau)) return PACE_ERR_UNSUPPORTED;
   pool->dev.adaptive = std::isfinite(tau) ? 1 : 0;
   pool->dev.tau2 = pool->dev.adaptive ? tau * tau : INFINITY;
+  return PACE_OK;
+}
+
+pace_status pace_set_commit_engine(pace_pool* pool, int32_t engine) {
+  if (!pool || (engine != PACE_COMMIT_MMA && engine != PACE_COMMIT_TCGEN05)) return PACE_ERR_INVALID_ARG;
+  if (engine == PACE_COMMIT_TCGEN05 && !(pool->maps_ok && pace::commit_tc_supported(pool->dev)))
+    return PACE_ERR_UNSUPPORTED;
+  pool->commit_engine = engine;
   return PACE_OK;
 }
 

@@ -100,6 +100,14 @@ __device__ __forceinline__ void stsm_trans_b8(uint32_t row_addr, uint32_t v) {
   asm volatile("stmatrix.sync.aligned.m16n8.x1.trans.shared.b8 [%0], {%1};" ::"r"(row_addr), "r"(v) : "memory");
 }
 
+// Four 8 x 16-byte matrices at once: threads 8m .. 8m + 7 give the row
+// addresses of matrix m, register m holds that matrix's bytes as above.
+__device__ __forceinline__ void stsm_trans_b8_x4(uint32_t row_addr, uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3) {
+  asm volatile("stmatrix.sync.aligned.m16n8.x4.trans.shared.b8 [%0], {%1, %2, %3, %4};" ::"r"(row_addr), "r"(v0),
+               "r"(v1), "r"(v2), "r"(v3)
+               : "memory");
+}
+
 // ---- bulk and tensor stores (shared -> global) ------------------------------
 __device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
@@ -117,6 +125,28 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed group has completed (writes visible).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// ---- waits --------------------------------------------------------------------
+// Wait for phase `parity` of `bar`, letting the hardware suspend the thread
+// between tests (up to 1 ms per test) instead of spinning; false and
+// PACE_FLAG_TIMEOUT once kWaitLimitNs of global time have passed.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t* flags) {
+  const uint64_t t0 = global_ns();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
+        : "memory");
+    if (ok) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      if (flags) atomicOr(flags, PACE_FLAG_TIMEOUT);
+      return false;
+    }
+  }
+}
 
 // ---- mbarrier arrive and named barriers --------------------------------------
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {

@@ -25,12 +25,15 @@ def _pace():
 
 
 def _run_periods(w, periods: int, seed: int = 0, warm_tokens: int = None, check_commit=True,
-                 random_init=False):
-    """Teacher-forced periods over every head of a small pool."""
+                 random_init=False, engine=None):
+    """Teacher-forced periods over every head of a small pool (commit engine:
+    the pool's default unless given)."""
     pace = _pace()
     bits = pace_synth.head_bits(w, seed)
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype)
+    if engine is not None:
+        pool.set_commit_engine(engine)
     if random_init:
         S0 = pace_synth.random_state(len(heads), w.d_v, w.d_k, seed=seed).numpy()
         state, _ = orc.PoolState.from_fp32(S0, [bits[h] for _, h in heads], w.axis)
