@@ -229,13 +229,22 @@ def run_reference(args, rank: int, world: int):
         samples.append(oracle_sample_rate(w, bits, 1, args.seed))
     val = statistics.median(s["value"] for s in samples)
     base = samples[0]
-    per_step_ms = 1000.0 * w.B * w.H * w.P / val
+    # each timed step is one whole sequence (all H heads) for one period: the
+    # time of that sample, not of the full pool; the rate is per head-token
+    sample_ms = 1000.0 * w.H * w.P / val
     line = {
         "impl": "reference", "metric": "decode head-tokens/s (B x H heads, 4-bit state, P=%d)" % w.P,
         "value": val, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": sample_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, bits),
+        "config": dict(workload_config(w, bits, state_bytes_of(w, bits)),
+                       parallelism=f"{world} independent pools (no collective)",
+                       int8_head_choice="seeded",
+                       int8_head_list=[h for h in range(w.H) if bits[h] == 8],
+                       seq_tokens_per_s=val / w.H),
+        "step_sample": f"one sequence (all {w.H} heads) for one period of P={w.P} tokens per step",
+        "extrapolated_from_heads": w.H,
+        "full_pool_ms_per_period_at_this_rate": 1000.0 * w.B * w.H * w.P / val,
         "cpu_baseline": dict(base, value=val),
         "e2e": {"value": val, "unit": "head-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -244,6 +253,14 @@ def run_reference(args, rank: int, world: int):
 
 
 L2_BYTES = 126 * 1024 * 1024
+
+
+def state_bytes_of(w, bits):
+    """Bytes of the pool's state region (records of codes + FP16 scales, each
+    padded to 16 bytes), by the layout include/pace.h documents."""
+    groups = w.d_k if w.axis == "col" else w.d_v
+    rec = [(w.d_v * w.d_k * b // 8 + 2 * groups + 15) // 16 * 16 for b in bits]
+    return w.B * ((sum(rec) + 15) // 16 * 16)
 
 
 def workload_config(w, bits, state_bytes=None):
@@ -526,6 +543,7 @@ def run_pace(args, rank: int, world: int):
                                              if args.bits_from_gates else "seeded"),
                            int8_head_list=[h for h in range(w.H) if bits[h] == 8],
                            seq_tokens_per_s=value / w.H),
+            "buffer_bytes": int(pool.buffer.numel()),
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                          "frac": ach / hbm, "traffic": traffic, "kernel": dominant,
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6.65 TB/s"},
@@ -718,7 +736,9 @@ def run_e2e(args, pace, pool, w, toks, outs, stream, world, dev, stag=None):
     from bit_recurrent_state_pace_b200.ranks import aggregate_rate
     return {"value": aggregate_rate(w.B * w.H * P * args.e2e_steps, world, ms),
             "unit": "head-tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+            "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+            # host-buffer decode is bound by the host link: the rates it reached
+            "h2d_gbs": h2d * args.e2e_steps / ms / 1e6, "d2h_gbs": d2h * args.e2e_steps / ms / 1e6}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing

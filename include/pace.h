@@ -120,7 +120,11 @@ pace_status pace_pool_bytes(const pace_pool_desc* desc, size_t* state_bytes,
                             size_t* buffer_bytes, size_t* aux_bytes);
 
 /*
- * Bind caller-owned device regions to a new pool.  Copies the descriptor
+ * Bind caller-owned device regions to a new pool: the per-request state pool
+ * whose size sets how many sequences can be served ([P4] TL;DR: 4-bit states
+ * fit about four times the concurrency of FP16 ones; [P2] "Periodic
+ * Rounding": the state, its small token buffer and the per-period factors).
+ * Copies the descriptor
  * (head_bits included), computes the record layout, and zeroes aux (all
  * buffers empty, status clear) with cudaMemsetAsync on `stream`.  The state
  * contents are the caller's (fill them with pace_pool_load or by writing
@@ -252,12 +256,18 @@ pace_status pace_quantize(const float* S, int64_t n_mats, int32_t d_k, int32_t d
                           int32_t bits, int32_t scale_axis, void* codes, uint16_t* scales,
                           uint32_t* d_flags, void* stream);
 
-/* Inverse of pace_quantize: S = float(code) * float(scale), exact in fp32. */
+/* Inverse of pace_quantize ([P2] "Channel-Aligned Encoding": each state entry
+ * is its code times its channel's scale): S = float(code) * float(scale),
+ * exact in fp32. */
 pace_status pace_dequantize(const void* codes, const uint16_t* scales, int64_t n_mats,
                             int32_t d_k, int32_t d_v, int32_t bits, int32_t scale_axis,
                             float* S, void* stream);
 
-/* Synchronise `stream`, then read the pool's device status word into *flags.
+/* The conditions the kernels detect on the device are kept as bits of one
+ * status word (the encoder's non-finite and clamped groups of [P2]
+ * "Channel-Aligned Encoding", a decode into a full buffer of [P2] "Periodic
+ * Rounding", a bounded wait that gave up).
+ * Synchronise `stream`, then read the pool's device status word into *flags.
  * Returns PACE_ERR_DEVICE_FLAGS if any bit is set, PACE_OK otherwise. */
 pace_status pace_pool_status(pace_pool* pool, void* stream, uint32_t* flags);
 
@@ -294,7 +304,11 @@ pace_status pace_gdn_step_bf16(uint16_t* S, const void* q, const void* k, const 
  * copies wait for the work already on `stream`, except when d_staging is the
  * buffer of this pool's previous call: then each slot is refilled as soon as
  * that call's last output copy from it is done, so consecutive calls keep
- * the copy engines busy.  The three streams must be distinct
+ * the copy engines busy.  That reuse is recognised by the pointer value
+ * alone: a caller that frees the staging buffer and gets the same address
+ * back for other work must order that work after this call (e.g. on
+ * `stream`), since the next call's input copies start without waiting for
+ * `stream`.  The three streams must be distinct
  * (PACE_ERR_INVALID_ARG otherwise, as for a NULL or unaligned d_staging or a
  * NULL input).  Enqueues only; `stream` completes after the last output
  * copy.  Not safe to call concurrently on one pool.  This host-buffer entry

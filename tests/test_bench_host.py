@@ -29,6 +29,15 @@ def test_reference_arm_prints_the_contract_line():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    # the same config keys as the GPU arm prints, with the pool's state size
+    for key in ("workload", "B", "H", "P", "int8_heads", "l2", "parallelism", "int8_head_choice",
+                "int8_head_list", "seq_tokens_per_s"):
+        assert key in line["config"], key
+    assert "larger than L2" in line["config"]["l2"]
+    # ms_per_step is the time of the sample actually run (one sequence, one period)
+    H, P = line["config"]["H"], line["config"]["P"]
+    assert abs(line["ms_per_step"] - 1000.0 * H * P / line["value"]) <= 1e-6 * line["ms_per_step"]
+    assert line["extrapolated_from_heads"] == H
 
 
 def test_profiles_hold_traffic_for_the_current_kernel_sources():

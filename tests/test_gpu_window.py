@@ -119,6 +119,9 @@ def _run(w, T, seed=0, e4m3_rows=False):
     ("mixed_4_8", dict(axis="row")),
     ("gdn_layer_4b", dict(d_k=64, d_v=64, P=5, io_dtype="f32", outliers=False)),
     ("mixed_4_8", dict(d_k=32, d_v=32, P=16)),
+    # 1024-byte fp32 rows: the shift moves two 16-byte pieces per lane, and
+    # P = 6 leaves a partial group of four rows
+    ("gdn_layer_4b", dict(P=6, io_dtype="f32", outliers=False)),
 ])
 def test_window_against_oracle(name, over, e4m3_rows):
     """The window's pairs as E4M3 bytes (the pool's buffer_e4m3 layout) or as
