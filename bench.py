@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16-state comparison path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-period-sweep", action="store_true",
+                    help="skip the period sweep (B=512, H=32, P in 1,2,4,8,16 with fp32-trajectory drift)")
+    ap.add_argument("--sweep-tokens", type=int, default=1024, help="decode tokens per period in the sweep")
     ap.add_argument("--cpu-sample-slots", type=int, default=32)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--schedule", choices=["staggered", "lockstep"], default="lockstep",
@@ -531,6 +534,13 @@ def run_pace(args, rank: int, world: int):
                    "status": pool.status()}
         del pin, po
 
+    # ---- period sweep on its own workload (one GPU only: it has no collective
+    #      and would only lengthen a multi-rank run)
+    sweep = None
+    if world == 1 and not args.no_period_sweep and stag is None:
+        del toks, outs
+        sweep = run_period_sweep(args, pace, dev, mk)
+
     if rank == 0:
         line = {
             "metric": "decode head-tokens/s (B x H heads, 4-bit state, P=%d)" % P,
@@ -568,9 +578,126 @@ def run_pace(args, rank: int, world: int):
             "prefill": prefill,
             "adaptive": adaptive,
             "window": window,
+            "period_sweep": sweep,
             "cpu_baseline": cpu_base,
         }
         print(json.dumps(line), flush=True)
+
+
+def run_period_sweep(args, pace, dev, mk):
+    """The period-sweep workload (B=512, H=32, d=128, all INT4, outlier value
+    channels, bf16 io) for each P in {1, 2, 4, 8, 16}: throughput, per-kernel
+    HBM GB/s, and the drift of the outputs from an unquantised fp32 trajectory
+    run on the same tokens.
+
+    Every P starts from the same pool: the 512-token fp32 warm-up state,
+    encoded.  The fp32 trajectory (pace_gdn_step_f32) starts from that
+    encoded state, dequantised, so that what it measures is the rounding
+    during decode, not the one initial encode they share.  Drift of head
+    (b, h) at token t: ||o - o_fp32||_inf / ||o_fp32||_inf; mean and max over
+    the B x H heads at a few horizons."""
+    import torch
+    import pace_synth
+
+    w0 = pace_synth.workload("period_sweep")
+    T = args.sweep_tokens
+    bits = pace_synth.head_bits(w0, args.seed)
+    BH = w0.B * w0.H
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    io_code = pace.PACE_IO_BF16 if w0.io_dtype == "bf16" else pace.PACE_IO_F32
+    horizons = [t for t in (8, 16, 64, 256, 1024, 4096) if t <= T]
+    if T not in horizons:
+        horizons.append(T)
+
+    S = torch.zeros(BH, w0.d_v, w0.d_k, dtype=torch.float32, device=dev)
+    for t in range(w0.warmup):
+        inp = pace_synth.token_inputs(w0, t, seed=args.seed, device=dev, phase="warmup")
+        pace.pace_gdn_step_f32(S, inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                               io_code, None, BH, w0.d_k, w0.d_v)
+    toks = [pace_synth.token_inputs(w0, t, seed=args.seed, device=dev) for t in range(T)]
+
+    # the unquantised trajectory from the encoded start
+    pool = pace.PacePool(w0.B, w0.H, w0.d_k, w0.d_v, 1, bits, axis=w0.axis, io=w0.io_dtype, device=dev)
+    pool.load(S)
+    S_ref = pool.export().view(BH, w0.d_v, w0.d_k).contiguous()
+    del pool
+    o = torch.empty(w0.B, w0.H, w0.d_v, dtype=torch.float32, device=dev)
+    ref = {}
+    for t in range(T):
+        x = toks[t]
+        pace.pace_gdn_step_f32(S_ref, x["q"], x["k"], x["v"], x["alpha"], x["beta"], io_code, o,
+                               BH, w0.d_k, w0.d_v)
+        if t + 1 in horizons:
+            ref[t + 1] = o.clone()
+    del S_ref
+    hbm = measured_peaks()[0]
+
+    def drift(out, r):
+        num = (out - r).abs().amax(-1)
+        den = r.abs().amax(-1).clamp_min(1e-30)
+        e = (num / den).flatten()
+        return {"mean": float(e.mean()), "max": float(e.max())}
+
+    rows = []
+    for P in pace_synth.PERIOD_SWEEP:
+        w = w0.replace(P=P)
+        pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, P, bits, axis=w.axis, io=w.io_dtype, device=dev)
+        pool.load(S)
+        dev_ev = [(mk(), mk()) for _ in range(T)]
+        com_ev = [(mk(), mk()) for _ in range(T // P)]
+        got = {}
+        torch.cuda.synchronize()
+        a, b = mk(), mk()
+        a.record(stream)
+        for t in range(T):
+            x = toks[t]
+            dev_ev[t][0].record(stream)
+            pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], o, sp)
+            dev_ev[t][1].record(stream)
+            if t + 1 in horizons:
+                got[t + 1] = o.clone()
+            if (t + 1) % P == 0:
+                c = com_ev[(t + 1) // P - 1]
+                c[0].record(stream)
+                pace.pace_commit_period(pool.handle, sp)
+                c[1].record(stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        status = pool.status()
+        dec_ms = [e0.elapsed_time(e1) for e0, e1 in dev_ev]
+        com_ms = [e0.elapsed_time(e1) for e0, e1 in com_ev]
+        dec_bytes = [alg_bytes(w, bits, t % P + 1)[0] for t in range(T)]
+        com_bytes = alg_bytes(w, bits, P)[1]
+        kern_ms = sum(dec_ms) + sum(com_ms)
+        dec_gbs = sum(dec_bytes) / (sum(dec_ms) * 1e-3) / 1e9
+        com_gbs = com_bytes * len(com_ms) / (sum(com_ms) * 1e-3) / 1e9 if com_ms else None
+        rows.append({
+            "P": P, "tokens": T,
+            "value": BH * T / (kern_ms * 1e-3), "unit": "head-tokens/s",
+            "ms_per_token": kern_ms / T,
+            "wall_ms": a.elapsed_time(b),
+            "decode": {"avg_ms": sum(dec_ms) / T, "achieved_gbs": dec_gbs, "frac_of_peak": dec_gbs / hbm},
+            "commit": {"launches": len(com_ms), "avg_ms": sum(com_ms) / max(1, len(com_ms)),
+                       "achieved_gbs": com_gbs, "frac_of_peak": com_gbs / hbm if com_gbs else None},
+            "hbm_gbs_per_token": (sum(dec_bytes) + com_bytes * len(com_ms)) / (kern_ms * 1e-3) / 1e9,
+            "drift": {str(h): drift(got[h], ref[h]) for h in horizons},
+            "device_status": status,
+        })
+        del pool, got
+    del toks, S, ref
+    torch.cuda.synchronize()
+    return {
+        "workload": f"period_sweep: B={w0.B} H={w0.H} d_k={w0.d_k} d_v={w0.d_v}, all INT4, "
+                    f"{w0.axis} scales, {w0.io_dtype} io, {w0.warmup}-token fp32 warm-up, {T} decode tokens",
+        "state_bytes": state_bytes_of(w0, bits),
+        "l2": "state pool 138 MB, near the 126 MB L2: no flush; part of the traffic is served from L2",
+        "drift_metric": "per head ||o - o_fp32||_inf / ||o_fp32||_inf at token t (mean, max over heads); "
+                        "o_fp32 from pace_gdn_step_f32 started at the encoded warm state, dequantised",
+        "time": "sum of per-launch CUDA-event durations (value); wall_ms includes the output copies "
+                "taken at the horizons",
+        "rows": rows,
+    }
 
 
 def gram_norm2(pool, w):

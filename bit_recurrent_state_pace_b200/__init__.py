@@ -20,6 +20,7 @@ import torch
 __all__ = [
     "PaceError", "lib", "LIB_PATH",
     "PACE_SCALE_COL", "PACE_SCALE_ROW", "PACE_IO_BF16", "PACE_IO_F32",
+    "PACE_OK", "PACE_ERR_INVALID_ARG", "PACE_ERR_UNSUPPORTED", "PACE_ERR_CUDA", "PACE_ERR_DEVICE_FLAGS",
     "PACE_FLAG_NONFINITE", "PACE_FLAG_SCALE_OVERFLOW", "PACE_FLAG_BUFFER_FULL", "PACE_FLAG_TIMEOUT",
     "PACE_FILL_COMMIT",
     "pace_pool_bytes", "pace_init_pool", "pace_destroy_pool", "pace_pool_layout",
@@ -28,7 +29,7 @@ __all__ = [
     "pace_select_head_bits", "pace_prefill", "pace_prefill_range", "pace_host_staging_bytes",
     "pace_decode_host", "pace_set_commit_threshold", "pace_window_scratch_bytes", "pace_window_step",
     "pace_window_step_static", "PACE_WINDOW_STATIC_SCRATCH_BYTES", "pace_set_commit_engine",
-    "PACE_COMMIT_MMA", "PACE_COMMIT_TCGEN05",
+    "PACE_COMMIT_MMA", "PACE_COMMIT_TCGEN05", "pace_debug_wait_fault",
     "pace_quantize", "pace_dequantize", "pace_pool_status", "pace_pool_clear_status",
     "pace_gdn_step_f32", "pace_gdn_step_bf16", "pace_status_string", "pace_version",
     "PacePool",
@@ -45,7 +46,7 @@ PACE_FLAG_TIMEOUT = 0x8
 PACE_FILL_COMMIT = 0x100
 PACE_WINDOW_STATIC_SCRATCH_BYTES = 8 << 20
 PACE_COMMIT_MMA, PACE_COMMIT_TCGEN05 = 0, 1
-PACE_OK, PACE_ERR_DEVICE_FLAGS = 0, 4
+PACE_OK, PACE_ERR_INVALID_ARG, PACE_ERR_UNSUPPORTED, PACE_ERR_CUDA, PACE_ERR_DEVICE_FLAGS = 0, 1, 2, 3, 4
 
 
 class PaceError(RuntimeError):
@@ -85,6 +86,7 @@ def _load():
         "pace_host_staging_bytes": [P, Sp],
         "pace_set_commit_threshold": [P, ctypes.c_float],
         "pace_set_commit_engine": [P, I32],
+        "pace_debug_wait_fault": [P, ctypes.c_uint64, ctypes.c_uint32],
         "pace_window_scratch_bytes": [P, Sp],
         "pace_window_step": [P, P, P, P, P, P, F32p, P, P],
         "pace_window_step_static": [P, P, P, P, P, P, F32p, P],
@@ -220,6 +222,10 @@ def pace_set_commit_threshold(handle: int, tau: float) -> None:
 
 def pace_set_commit_engine(handle: int, engine: int) -> None:
     _check("pace_set_commit_engine", lib.pace_set_commit_engine(handle, int(engine)))
+
+
+def pace_debug_wait_fault(handle: int, wait_limit_ns: int, extra_tx_bytes: int) -> None:
+    _check("pace_debug_wait_fault", lib.pace_debug_wait_fault(handle, int(wait_limit_ns), int(extra_tx_bytes)))
 
 
 def pace_host_staging_bytes(handle: int) -> int:

@@ -449,9 +449,7 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       const float a0 = m0 * down, a1 = m1 * down;
       const GroupScale s0 = group_scale(a0, isfinite(a0), qmax, p.flags);
       const GroupScale s1 = group_scale(a1, isfinite(a1), qmax, p.flags);
-      const bool bad = !isfinite(a0) || !isfinite(a1) ||
-                       (s0.bits == 0x7BFF && a0 / qmax > 65504.f) ||
-                       (s1.bits == 0x7BFF && a1 / qmax > 65504.f);
+      const bool bad = !fast_encode_ok(a0, s0, qmax) || !fast_encode_ok(a1, s1, qmax);
       rsc[i0] = s0.bits;
       rsc[i1] = s1.bits;
       sm.qf[i0] = s0.sf > 0.f ? __frcp_rn(s0.sf) : 0.f;
@@ -472,7 +470,7 @@ __device__ bool commit_head(const PoolDev& p, int head, Smem<D, BF16, PMAX>& sm,
       rsc[j] = s.bits;
       sm.qf[j] = s.sf > 0.f ? __frcp_rn(s.sf) : 0.f;
       sm.sfv[j] = s.sf;
-      if (!isfinite(a) || (s.bits == 0x7BFF && a / qmax > 65504.f)) slow_flag = 1;
+      if (!fast_encode_ok(a, s, qmax)) slow_flag = 1;
     }
     __syncthreads();
   }

@@ -591,7 +591,7 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
     const GroupScale gs = group_scale(amax, isfinite(amax), qmax, p.flags);
     sf = gs.sf;
     qf = gs.sf > 0.f ? __frcp_rn(gs.sf) * down : 0.f;
-    bad = !isfinite(amax) || (gs.bits == 0x7BFF && amax / qmax > 65504.f) || !(qf < INFINITY);
+    bad = !fast_encode_ok(amax, gs, qmax) || !(qf < INFINITY);
     reinterpret_cast<uint16_t*>(stg + 16384)[chan_of<BITS>(pos)] = gs.bits;
   }
   const bool slow = __any_sync(FULL, bad);

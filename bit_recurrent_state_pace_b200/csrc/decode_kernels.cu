@@ -636,7 +636,7 @@ __device__ __forceinline__ void issue_stage(const PoolDev& p, int head, int fill
   const uint32_t kv_bytes = rows ? (uint32_t)fill * 2 * RB : 0u;
   const uint32_t bytes = 3 * IO + 2 * D + (rows ? kv_bytes + p.ab_stride + p.gram_stride : 0u);
   fence_proxy_async_smem();
-  mbar_arrive_expect_tx(bar, bytes);
+  mbar_arrive_expect_tx(bar, bytes + p.dbg_extra_tx);
   tma_load_1d(stg + ST::Q, reinterpret_cast<const uint8_t*>(q) + (size_t)head * IO, IO, bar);
   tma_load_1d(stg + ST::K, reinterpret_cast<const uint8_t*>(k) + (size_t)head * IO, IO, bar);
   tma_load_1d(stg + ST::V, reinterpret_cast<const uint8_t*>(v) + (size_t)head * IO, IO, bar);
@@ -702,12 +702,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       f_cur = f_nxt;
       f_nxt = it + 2 * W < n_heads ? p.fill[head_in_order(p, it + 2 * W, sp.b0, sp.nb)] : 0;
     }
-    const bool ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, lane == 0 ? p.flags : nullptr);
+    const bool ok =
+        mbar_wait_bounded(&bar[s], (parity >> s) & 1u, lane == 0 ? p.flags : nullptr, p.wait_limit_ns);
     parity ^= 1u << s;
     if (!__all_sync(FULL, ok)) {
-      // a copy did not land in time: let the other stage's copy finish (bounded)
-      // before this warp stops using its shared memory
-      if (NS == 2 && nh >= 0) mbar_wait_bounded(&bar[s ^ 1], (parity >> (s ^ 1)) & 1u, nullptr);
+      // a copy did not land in time: this head's output row is NaN; let the
+      // other stage's copy finish (bounded) before the warp stops using its
+      // shared memory
+      for (int i = lane; i < D; i += 32) o[(size_t)head * D + i] = __int_as_float(0x7fc00000);
+      if (NS == 2 && nh >= 0) mbar_wait_bounded(&bar[s ^ 1], (parity >> (s ^ 1)) & 1u, nullptr, p.wait_limit_ns);
       return;
     }
     const uint8_t* stg = stages + s * ST::BYTES;

@@ -41,6 +41,18 @@ __device__ __forceinline__ GroupScale group_scale(float amax, bool finite, int q
   return r;
 }
 
+// The fast encode of the update kernels (x * (1 / s16) rounded by a
+// magic-number add, no clamp) gives the exact encoder's codes, up to exact
+// ties, when every |x| <= amax has |x / s16| < qmax + 1/2.  That holds when
+// s16 rounds amax / qmax to a normal fp16 (relative error <= 2^-11) but can
+// fail for a scale in the fp16 subnormal range or raised to 2^-24 (amax far
+// below 1e-4); such groups, and non-finite ones, take the exact encoder.
+__device__ __forceinline__ bool fast_encode_ok(float amax, const GroupScale& gs, int qmax) {
+  if (!isfinite(amax)) return false;
+  if (gs.sf == 0.f) return true;   // all-zero group: every code is 0
+  return amax * __frcp_rn(gs.sf) < (float)qmax + 0.25f;
+}
+
 __device__ __forceinline__ int encode_value(float x, float sf, int qmax) {
   if (sf == 0.f) return 0;
   float c = rintf(__fdiv_rn(x, sf));

@@ -35,6 +35,8 @@ struct PoolDev {
   float tau2;                         // commit threshold squared (+inf: fixed period)
   int32_t adaptive;                   // tau2 finite
   int32_t row8;                       // buffered k, v rows are E4M3 bytes
+  uint32_t dbg_extra_tx;              // 0; > 0 only under pace_debug_wait_fault
+  uint64_t wait_limit_ns;             // bound of the decode's mbarrier waits
 };
 
 // Bytes per buffered k or v element.

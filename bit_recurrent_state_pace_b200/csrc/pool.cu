@@ -6,6 +6,7 @@
 
 #include "commit_tc.cuh"
 #include "pace_internal.cuh"
+#include "tma.cuh"
 #include "window.cuh"
 
 struct pace_pool {
@@ -178,6 +179,8 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
   dv.tau2 = INFINITY;
   dv.adaptive = 0;
   dv.row8 = desc->buffer_e4m3;
+  dv.dbg_extra_tx = 0;
+  dv.wait_limit_ns = pace::kWaitLimitNs;
   for (int h = 0; h < desc->num_heads; ++h) {
     dv.rec_off[h] = (uint32_t)L.rec_off[h];
     dv.bits[h] = desc->head_bits[h];
@@ -259,6 +262,23 @@ pace_status pace_set_commit_engine(pace_pool* pool, int32_t engine) {
   if (engine == PACE_COMMIT_TCGEN05 && !(pool->maps_ok && pace::commit_tc_supported(pool->dev)))
     return PACE_ERR_UNSUPPORTED;
   pool->commit_engine = engine;
+  return PACE_OK;
+}
+
+pace_status pace_debug_wait_fault(pace_pool* pool, uint64_t wait_limit_ns, uint32_t extra_tx_bytes) {
+  if (!pool) return PACE_ERR_INVALID_ARG;
+  if (extra_tx_bytes == 0 && wait_limit_ns == 0) {   // back to the defaults
+    pool->dev.dbg_extra_tx = 0;
+    pool->dev.wait_limit_ns = pace::kWaitLimitNs;
+    return PACE_OK;
+  }
+  if (wait_limit_ns < 1000 || wait_limit_ns > pace::kWaitLimitNs || extra_tx_bytes > 16 ||
+      (extra_tx_bytes & 15u) != 0)
+    return PACE_ERR_INVALID_ARG;
+  if (extra_tx_bytes > 0 && (wait_limit_ns > 10000000ull || pool->dev.B * pool->dev.H != 1))
+    return PACE_ERR_INVALID_ARG;
+  pool->dev.dbg_extra_tx = extra_tx_bytes;
+  pool->dev.wait_limit_ns = wait_limit_ns;
   return PACE_OK;
 }
 

@@ -508,9 +508,7 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       sm.qf[i1] = s1.sf > 0.f ? __frcp_rn(s1.sf) : 0.f;
       sm.sfv[i0] = s0.sf;
       sm.sfv[i1] = s1.sf;
-      if (!isfinite(a0) || !isfinite(a1) || (s0.bits == 0x7BFF && a0 / qmax > 65504.f) ||
-          (s1.bits == 0x7BFF && a1 / qmax > 65504.f))
-        sm.slow = 1;
+      if (!fast_encode_ok(a0, s0, qmax) || !fast_encode_ok(a1, s1, qmax)) sm.slow = 1;
     }
   }
   __syncthreads();
@@ -523,7 +521,7 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       rsc[j] = s.bits;
       sm.qf[j] = s.sf > 0.f ? __frcp_rn(s.sf) : 0.f;
       sm.sfv[j] = s.sf;
-      if (!isfinite(a) || (s.bits == 0x7BFF && a / qmax > 65504.f)) sm.slow = 1;
+      if (!fast_encode_ok(a, s, qmax)) sm.slow = 1;
     }
     __syncthreads();
   }

@@ -275,6 +275,25 @@ pace_status pace_pool_status(pace_pool* pool, void* stream, uint32_t* flags);
 pace_status pace_pool_clear_status(pace_pool* pool, void* stream);
 
 /*
+ * Debug only: exercise the bounded waits of pace_decode_step.  No passage of
+ * the pages corresponds; it tests the failure detection of the status word
+ * (PACE_FLAG_TIMEOUT).  The decode stages each head's inputs with bulk
+ * copies that complete on an mbarrier, and its warps wait for that barrier
+ * for at most a fixed time (2 s by default) before giving up.
+ *  wait_limit_ns:   that bound, 1000 .. 2e9 ns.
+ *  extra_tx_bytes:  0 or 16.  With 16, every stage's barrier expects 16
+ *    bytes more than its copies bring: every copy still lands (nothing is
+ *    left in flight), the barrier never completes, each warp's wait runs
+ *    out after wait_limit_ns, the head's output row is NaN, nothing is
+ *    buffered, and PACE_FLAG_TIMEOUT is set.  Allowed only on a pool of
+ *    one head (B = H = 1) with wait_limit_ns <= 1e7.
+ * (0, 0) restores the defaults.  Out-of-range values are
+ * PACE_ERR_INVALID_ARG and change nothing.  Host-only; applies to launches
+ * enqueued after the call.
+ */
+pace_status pace_debug_wait_fault(pace_pool* pool, uint64_t wait_limit_ns, uint32_t extra_tx_bytes);
+
+/*
  * Unquantised comparison paths (not PACE; used for the fp32 warm-up prefill,
  * the drift reference trajectory and the bf16-state throughput comparison).
  * One token of the rule above for n independent heads, state updated in

@@ -54,16 +54,21 @@ def test_empty_slot_ranges_are_noops():
         assert torch.equal(a, b)
 
 
-def _teacher_forced_period(w, edit, seed=0):
-    """One period from a random stored state with the token inputs changed by
-    edit(inputs) (device tensors), against the oracle; returns (outputs, the
-    oracle's committed state, the GPU's codes and scales)."""
+def _teacher_forced_period(w, edit, seed=0, state_edit=None, engine=None):
+    """One period from a random stored state (changed by state_edit(S0) when
+    given) with the token inputs changed by edit(inputs) (device tensors),
+    against the oracle; returns (outputs, the oracle's committed state, the
+    GPU's codes and scales)."""
     pace = _pace()
     bits = pace_synth.head_bits(w, seed)
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     S0 = pace_synth.random_state(len(heads), w.d_v, w.d_k, seed=seed).numpy()
+    if state_edit is not None:
+        S0 = state_edit(S0)
     state, _ = orc.PoolState.from_fp32(S0, [bits[h] for _, h in heads], w.axis)
     pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype)
+    if engine is not None:
+        pool.set_commit_engine(engine)
     pu.load_state(pool, heads, state)
     toks, outs = [], []
     for t in range(w.P):
@@ -127,3 +132,40 @@ def test_alpha_one_beta_zero_keeps_the_state():
     for i in range(w.B * w.H):
         assert np.array_equal(gc[i], st.codes[i])
         assert np.array_equal(gs[i].view(np.uint16), st.scales[i].view(np.uint16))
+
+
+@pytest.mark.parametrize("axis,engine", [("col", "mma"), ("col", "tcgen05"), ("row", "mma")])
+@pytest.mark.parametrize("bits8", [False, True])
+def test_group_scale_in_the_fp16_subnormal_range(axis, engine, bits8):
+    """A group whose values are a few 2^-24: its stored FP16 scale is the
+    subnormal 2^-23, and after one period of decay with no writes
+    (gamma_P = 0.7346) the new absmax / qmax = 1.47 * 2^-24 rounds down to the
+    scale 2^-24.  The largest |x / s| is then about 10.3 (INT4) / 186 (INT8),
+    so the encoder clamps codes at qmax; every other group keeps normal
+    scales.  The commit must give the oracle's clamped codes, not codes past
+    qmax."""
+    w = pace_synth.workload("gdn_layer_4b", B=2, H=2, P=4, axis=axis, outliers=False,
+                            int8_fraction=1.0 if bits8 else 0.0)
+    qmax = 127 if bits8 else 7
+    tiny = 2.0 * qmax * 2.0 ** -24          # absmax with amax / qmax = 2^-23 exactly
+
+    def state_edit(S0):
+        S0 = S0.copy()
+        for m in range(S0.shape[0]):
+            g = S0[m, :, 5] if axis == "col" else S0[m, 5, :]
+            g[:] = np.clip(g / np.abs(g).max(), -1.0, 1.0) * tiny
+        return S0.astype(np.float32)
+
+    def edit(x):
+        x["beta"] = torch.zeros_like(x["beta"])
+        x["alpha"] = torch.full_like(x["alpha"], 0.92578125)   # bf16; gamma_4 = 0.7346
+        return x
+
+    pace = _pace()
+    eng = pace.PACE_COMMIT_TCGEN05 if engine == "tcgen05" else pace.PACE_COMMIT_MMA
+    _, _, committed, (gc, gs), _ = _teacher_forced_period(w, edit, state_edit=state_edit, engine=eng)
+    for m in range(len(committed.codes)):
+        assert int(committed.scales[m].view(np.uint16)[5]) == 0x0001
+        assert int(np.abs(np.asarray(gc[m], np.int64)).max()) <= qmax
+        c = committed.codes[m]
+        assert int(np.abs(c[:, 5] if axis == "col" else c[5, :]).max()) == qmax
