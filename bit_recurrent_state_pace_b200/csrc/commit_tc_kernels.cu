@@ -127,12 +127,14 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
   return r;
 }
 
-// First head index >= from (stepping by step, below end) due for a commit, or
-// end.  The 32 lanes of the calling warp test 32 candidates at a time.
-__device__ __forceinline__ int next_due(const PoolDev& p, int from, int step, int end, int lane) {
+// First work index >= from (stepping by step, below end) whose head is due
+// for a commit, or end.  Work index i is head head_in_order(i): the 4-bit
+// heads of the span first, so that a CTA runs one code path at a time.  The
+// 32 lanes of the calling warp test 32 candidates at a time.
+__device__ __forceinline__ int next_due(const PoolDev& p, int from, int step, int end, int b0, int nb, int lane) {
   for (int base = from; base < end; base += 32 * step) {
-    const int hd = base + lane * step;
-    const unsigned m = __ballot_sync(FULL, hd < end && commit_due(p.fill[hd], p.P));
+    const int it = base + lane * step;
+    const unsigned m = __ballot_sync(FULL, it < end && commit_due(p.fill[head_in_order(p, it, b0, nb)], p.P));
     if (m) return base + (__ffs((int)m) - 1) * step;
   }
   return end;
@@ -140,14 +142,16 @@ __device__ __forceinline__ int next_due(const PoolDev& p, int from, int step, in
 
 // ---- producer: stage the heads due for a commit ------------------------------
 template <bool BF16, bool R8, int PMAX>
-__device__ void producer_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, int first, int end, int lane) {
+__device__ void producer_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, const Span& sp, int lane) {
   using C = TcCfg<BF16, R8, PMAX>;
   const uint32_t row = (uint32_t)C::ROWB;
-  int h = next_due(p, first, gridDim.x, end, lane);
+  const int end = sp.nb * p.H;
+  int it = next_due(p, (int)blockIdx.x, gridDim.x, end, sp.b0, sp.nb, lane);
   for (int k = 0;; ++k) {
     const int s = k % C::NST, r = k / C::NST;
     if (r > 0 && !bounded_wait(&sm.stage_empty[s], (uint32_t)((r - 1) & 1), p, &sm.abort)) return;
-    const bool have = __shfl_sync(FULL, (h < end && !aborted(&sm.abort)) ? 1 : 0, 0) != 0;
+    const bool have = __shfl_sync(FULL, (it < end && !aborted(&sm.abort)) ? 1 : 0, 0) != 0;
+    const int h = have ? head_in_order(p, it, sp.b0, sp.nb) : -1;
     if (lane == 0) {
       sm.stage_head[s] = have ? h : -1;
       if (have) {
@@ -168,7 +172,7 @@ __device__ void producer_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, int 
     }
     __syncwarp();
     if (!have) return;
-    h = next_due(p, h + gridDim.x, gridDim.x, end, lane);
+    it = next_due(p, it + gridDim.x, gridDim.x, end, sp.b0, sp.nb, lane);
   }
 }
 
@@ -692,7 +696,6 @@ __global__ void __launch_bounds__(TcCfg<BF16, R8, PMAX>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int first = sp.b0 * p.H + (int)blockIdx.x, end = (sp.b0 + sp.nb) * p.H;
   if (tid == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&sm.stage_full[s], 1);
@@ -725,7 +728,7 @@ __global__ void __launch_bounds__(TcCfg<BF16, R8, PMAX>::THREADS, 1)
   tc::fence_after_sync();
   const uint32_t tm = sm.taddr;
   if (warp == 0) {
-    producer_role<BF16, R8, PMAX>(p, sm, first, end, lane);
+    producer_role<BF16, R8, PMAX>(p, sm, sp, lane);
   } else if (warp == 1) {
     if (lane == 0) mma_role<BF16, R8, PMAX>(p, sm, tm);
     __syncwarp();
