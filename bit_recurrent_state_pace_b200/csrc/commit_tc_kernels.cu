@@ -66,8 +66,10 @@ struct TcCfg {
   static constexpr int FIXED = 2 * (TILE + STG + BXB + 2 * AUB) + 4096;
   static constexpr int NST_FIT = (kSmemLimit - 1024 - FIXED) / STAGE;
   static constexpr int NST = NST_FIT > 4 ? 4 : NST_FIT;  // staged heads
-  static constexpr int THREADS = 10 * 32;                 // producer, MMA, 4 converter, 4 epilogue warps
-  static constexpr int CONV0 = 2, EPI0 = 6;               // first converter / epilogue warp
+  static constexpr int NCONV = 8, NEPI = 8;               // converter / epilogue warps (two per TMEM quadrant)
+  static constexpr int THREADS = (2 + NCONV + NEPI) * 32; // producer, MMA, converters, epilogue
+  static constexpr int CONV0 = 2, EPI0 = 2 + NCONV;       // first converter / epilogue warp
+  static constexpr int NCT = 32 * NCONV, NET = 32 * NEPI; // converter / epilogue threads
 };
 
 template <bool BF16, bool R8, int PMAX>
@@ -84,7 +86,8 @@ struct alignas(1024) TcSmem {
   // epilogue, in a ring of four (the head k + 4 reuses the slot of head k)
   float fj[4][128];                    // epilogue factors gamma_n s_j 2^e, by tile position
   int meta_head[4], meta_e[4], meta_bits[4];
-  float red[2][4];                     // converter maxima of |U^| (two heads alternate)
+  float red[2][8];                     // converter maxima of |U^| (two heads alternate)
+  float emax[2][128];                  // epilogue column maxima of the two value-channel halves
   int stage_head[C::NST], stage_n[C::NST];
   uint64_t stage_full[C::NST], stage_empty[C::NST];
   uint64_t tile_full[2], x_full[2], bupd_full[2], acc_full[2], tmem_empty[2], drain;
@@ -127,17 +130,33 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
   return r;
 }
 
-// First work index >= from (stepping by step, below end) whose head is due
-// for a commit, or end.  Work index i is head head_in_order(i): the 4-bit
-// heads of the span first, so that a CTA runs one code path at a time.  The
-// 32 lanes of the calling warp test 32 candidates at a time.
-__device__ __forceinline__ int next_due(const PoolDev& p, int from, int step, int end, int b0, int nb, int lane) {
-  for (int base = from; base < end; base += 32 * step) {
-    const int it = base + lane * step;
-    const unsigned m = __ballot_sync(FULL, it < end && commit_due(p.fill[head_in_order(p, it, b0, nb)], p.P));
-    if (m) return base + (__ffs((int)m) - 1) * step;
+// The producer's walk over its work items (work index i is head
+// head_in_order(i): the 4-bit heads of the span first, so that a CTA runs one
+// code path at a time).  The warp reads the fill counters of 32 items at a
+// time and keeps the mask of the due ones, so each head costs one global
+// round trip per 32 items, and the fill of the chosen one comes with it.
+struct DueScan {
+  int base;        // work index of lane 0's item in the current window
+  unsigned mask;   // due items of the window not taken yet
+  int fill;        // this lane's fill counter in the window
+};
+__device__ __forceinline__ void due_window(const PoolDev& p, DueScan& d, int step, int end, int b0, int nb, int lane) {
+  const int it = d.base + lane * step;
+  d.fill = it < end ? p.fill[head_in_order(p, it, b0, nb)] : 0;
+  d.mask = __ballot_sync(FULL, it < end && commit_due(d.fill, p.P));
+}
+// Next due work index (and its fill), or end.
+__device__ __forceinline__ int next_due(const PoolDev& p, DueScan& d, int step, int end, int b0, int nb, int lane,
+                                        int* fill) {
+  while (d.mask == 0) {
+    d.base += 32 * step;
+    if (d.base >= end) return end;
+    due_window(p, d, step, end, b0, nb, lane);
   }
-  return end;
+  const int l = __ffs((int)d.mask) - 1;
+  d.mask &= d.mask - 1;
+  *fill = __shfl_sync(FULL, d.fill, l);
+  return d.base + l * step;
 }
 
 // ---- producer: stage the heads due for a commit ------------------------------
@@ -146,7 +165,11 @@ __device__ void producer_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, cons
   using C = TcCfg<BF16, R8, PMAX>;
   const uint32_t row = (uint32_t)C::ROWB;
   const int end = sp.nb * p.H;
-  int it = next_due(p, (int)blockIdx.x, gridDim.x, end, sp.b0, sp.nb, lane);
+  DueScan due;
+  due.base = (int)blockIdx.x;
+  due_window(p, due, gridDim.x, end, sp.b0, sp.nb, lane);
+  int fill = 0;
+  int it = due.base < end ? next_due(p, due, gridDim.x, end, sp.b0, sp.nb, lane, &fill) : end;
   for (int k = 0;; ++k) {
     const int s = k % C::NST, r = k / C::NST;
     if (r > 0 && !bounded_wait(&sm.stage_empty[s], (uint32_t)((r - 1) & 1), p, &sm.abort)) return;
@@ -156,7 +179,7 @@ __device__ void producer_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, cons
       sm.stage_head[s] = have ? h : -1;
       if (have) {
         const int hh = h % p.H, b = h / p.H;
-        sm.stage_n[s] = p.fill[h] & 0xff;
+        sm.stage_n[s] = fill & 0xff;
         const uint32_t rec_bytes = (uint32_t)record_bytes(C::D, C::D, p.bits[hh], C::D);
         const uint32_t kv_bytes = (uint32_t)p.P * row;
         const uint8_t* rec = p.state + (size_t)b * p.slot_stride + p.rec_off[hh];
@@ -172,7 +195,7 @@ __device__ void producer_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, cons
     }
     __syncwarp();
     if (!have) return;
-    it = next_due(p, it + gridDim.x, gridDim.x, end, sp.b0, sp.nb, lane);
+    it = next_due(p, due, gridDim.x, end, sp.b0, sp.nb, lane, &fill);
   }
 }
 
@@ -231,16 +254,16 @@ __device__ void mma_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uint32_t 
 // Codes of one staged record -> the f16 tile (exact values), [jh][i][64
 // positions] with 128-byte swizzling.  Each lane converts 16 channels of one
 // row per step; a quarter-warp covers two rows whose halves are swapped, so
-// its loads and its 16-byte stores each fall in distinct banks.  The eight
-// steps of a lane differ by constant offsets (the swizzle term depends only
-// on the row modulo 8, which is fixed per lane).
-template <int BITS>
+// its loads and its 16-byte stores each fall in distinct banks.  A warp
+// converts RPW rows in RPW / 4 steps, which differ by constant offsets (the
+// swizzle term depends only on the row modulo 8, which is fixed per lane).
+template <int BITS, int RPW>
 __device__ __forceinline__ void convert_codes(const uint8_t* rec, uint8_t* tile, int cw, int lane) {
   const uint32_t K64 = 0x64646464u;
   const __half2 off8 = __float2half2_rn(1032.f), off16 = __float2half2_rn(-72.f);
   const __half2 sixteenth = __float2half2_rn(0.0625f), off128 = __float2half2_rn(1152.f);
   const int qq = lane >> 3, r = (lane >> 2) & 1, mm = lane & 3;
-  const int i0 = 32 * cw + 2 * qq + r;               // row of step 0; step it adds 8 (it >> 1)
+  const int i0 = RPW * cw + 2 * qq + r;              // row of step 0; step it adds 8 (it >> 1)
   const int r7 = i0 & 7;
   // group of the even steps (m16 = 4 r + mm) and of the odd ones (m16 = 4 (1 - r) + mm)
   const int mA = 4 * r + mm, mB = 4 * (1 - r) + mm;
@@ -252,7 +275,7 @@ __device__ __forceinline__ void convert_codes(const uint8_t* rec, uint8_t* tile,
   const int cB0 = ((2 * (mB & 3)) ^ r7) << 4, cB1 = ((2 * (mB & 3) + 1) ^ r7) << 4;
   const int rstride = BITS == 4 ? 512 : 1024;         // 8 rows of codes
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
+  for (int it = 0; it < RPW / 4; ++it) {
     const bool odd = it & 1;
     const uint8_t* src = (odd ? srcB : srcA) + rstride * (it >> 1);
     uint8_t* dst = (odd ? dstB : dstA) + 1024 * (it >> 1);
@@ -296,14 +319,16 @@ __device__ __forceinline__ KeyExp key_exponents(const float* G, int P) {
 // The scaled keys of one head: B of X (rows s: hi, PMAX + s: lo of
 // s_j k_s[j] 2^exx) and A of the update (rows s and PMAX + s: k_s[j] 2^exk
 // in f16, and rows 2 PMAX + s: its low part for fp32 rows), by tile
-// position.  Thread ct owns the position pair 2 (ct % 64) + {0, 1} and half
-// of the tokens.  Tokens s >= n give zero rows.
+// position.  Thread ct (of the NCT converter threads) owns the position
+// pair 2 (ct % 64) + {0, 1} and a share NCT / 64 of the tokens.  Tokens
+// s >= n give zero rows.
 template <bool BF16, bool R8, int PMAX, int BITS>
 __device__ __forceinline__ void build_keys(const uint8_t* stage, uint8_t* bx, uint8_t* au, int n, KeyExp ex, int ct) {
   using C = TcCfg<BF16, R8, PMAX>;
   const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + code_bytes(C::D, C::D, BITS));
   const uint8_t* rows = stage + C::REC;
-  const int pp = ct & 63, s0 = (ct >> 6) * (PMAX / 2);
+  constexpr int SPT = PMAX / (C::NCT / 64);   // tokens per thread
+  const int pp = ct & 63, s0 = (ct >> 6) * SPT;
   const int j0 = chan_of<BITS>(2 * pp), j1 = chan_of<BITS>(2 * pp + 1);
   const float upx = pow2i(ex.exx), upk = pow2i(ex.exk);
   const float2 sx = make_float2(__half2float(__ushort_as_half(sc[j0])) * upx,
@@ -314,7 +339,7 @@ __device__ __forceinline__ void build_keys(const uint8_t* stage, uint8_t* bx, ui
   uint8_t* xb = bx + half * (C::NX * 128) + word;
   uint8_t* ab = au + half * (C::KU * 128) + word;
 #pragma unroll
-  for (int s = s0; s < s0 + PMAX / 2; ++s) {
+  for (int s = s0; s < s0 + SPT; ++s) {
     float2 kv = make_float2(0.f, 0.f);
     if (s < n) {
       kv.x = row_at<R8>(rows + s * C::ROWB, j0, BF16);
@@ -341,24 +366,27 @@ __device__ __forceinline__ void build_keys(const uint8_t* stage, uint8_t* bx, ui
 // R and U^ for one head, one TMEM lane (value channel i) per converter thread:
 // x_s from TMEM, r_s = v_s[i] - gamma_s x_s, U^[s][i] = sum_s' W[s][s'] r_s',
 // normalised by one power of two for the head, split hi + lo into row i of
-// the update's B.  Also the epilogue's per-position factors.  A head with
-// all PMAX tokens takes packed pair arithmetic over the factor rows; early
-// commits (n < PMAX) take guarded scalar loops.
+// the update's B.  The two converter warps of a TMEM lane quadrant split the
+// tokens s (each forms all of R).  Also the epilogue's per-position factors.
+// A head with all PMAX tokens takes packed pair arithmetic over the factor
+// rows; early commits (n < PMAX) take guarded scalar loops.
 template <bool BF16, bool R8, int PMAX>
 __device__ __forceinline__ void residual_update(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, const uint8_t* stage,
                                                 int bits, int t, int n, uint32_t tm, int k, int ct, int warp,
                                                 int lane) {
   using C = TcCfg<BF16, R8, PMAX>;
+  constexpr int H2 = PMAX / 2;                   // tokens per half
   const int m = k & 3;   // ring slot of this head
   const int P = p.P;
   const int qd = warp & 3, i = 32 * qd + lane;
+  const int sb = ((warp - C::CONV0) >> 2) * H2;  // this warp's tokens [sb, sb + H2)
   const float* G = reinterpret_cast<const float*>(stage + C::REC + C::KVB);
   const float* W = G;
   const float* gam = G + P * P;
   const KeyExp ex = key_exponents(G, P);
   const float xinv = pow2i(-ex.exx);
   const uint8_t* vrow = stage + C::REC + C::D * C::ESZ + i * C::ESZ;   // v_0[i]
-  float x[PMAX], r[PMAX], u[PMAX];
+  float x[PMAX], r[PMAX], u[H2];
   {
     uint32_t xa[16], xb[16];
     tc::ld_32x32b_x16(tm + ((uint32_t)(32 * qd) << 16) + 256u * t + 128u, xa);
@@ -377,7 +405,7 @@ __device__ __forceinline__ void residual_update(const PoolDev& p, TcSmem<BF16, R
     }
   }
   const bool full = n == PMAX && P == PMAX;
-  float um;
+  float um = 0.f;
   if (full) {
 #pragma unroll
     for (int s2 = 0; s2 < PMAX; s2 += 2) {
@@ -387,51 +415,51 @@ __device__ __forceinline__ void residual_update(const PoolDev& p, TcSmem<BF16, R
       r[s2] = rr.x;
       r[s2 + 1] = rr.y;
     }
-    float2 mu = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int s = 0; s < PMAX; ++s) {
+    for (int s = 0; s < H2; ++s) {
       float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < PMAX; c += 4) {
-        const float4 w4 = *reinterpret_cast<const float4*>(W + s * PMAX + c);
+        const float4 w4 = *reinterpret_cast<const float4*>(W + (sb + s) * PMAX + c);
         acc = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(r[c], r[c + 1]), acc);
         acc = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(r[c + 2], r[c + 3]), acc);
       }
       u[s] = acc.x + acc.y;
     }
-    um = 0.f;
 #pragma unroll
-    for (int s = 0; s < PMAX; s += 2) um = max3_nan(um, fabsf(u[s]), fabsf(u[s + 1]));
-    (void)mu;
+    for (int s = 0; s < H2; s += 2) um = max3_nan(um, fabsf(u[s]), fabsf(u[s + 1]));
   } else {
 #pragma unroll
     for (int s = 0; s < PMAX; ++s)
       r[s] = s < n ? row_at<R8>(vrow + s * C::ROWB, 0, BF16) - gam[s] * (x[s] * xinv) : 0.f;
-    um = 0.f;
 #pragma unroll
-    for (int s = 0; s < PMAX; ++s) {
+    for (int s = 0; s < H2; ++s) {
+      const int ss = sb + s;
       float a = 0.f;
 #pragma unroll
       for (int sp = 0; sp < PMAX; ++sp)
-        if (s < n && sp < n) a = fmaf(W[s * P + sp], r[sp], a);
+        if (ss < n && sp < n) a = fmaf(W[ss * P + sp], r[sp], a);
       u[s] = a;
       um = max_nan(um, fabsf(a));
     }
   }
-  // one exponent for the head's U^ (all 128 lanes feed one product)
+  // one exponent for the head's U^ (all 128 lanes and both halves feed one product)
 #pragma unroll
   for (int off = 16; off; off >>= 1) um = max_nan(um, __shfl_xor_sync(FULL, um, off));
   if (lane == 0) sm.red[k & 1][warp - C::CONV0] = um;
-  tc::named_sync(6, 128);
-  um = max3_nan(max_nan(sm.red[k & 1][0], sm.red[k & 1][1]), sm.red[k & 1][2], sm.red[k & 1][3]);
+  tc::named_sync(6, C::NCT);
+  um = 0.f;
+#pragma unroll
+  for (int w = 0; w < C::NCONV; ++w) um = max_nan(um, sm.red[k & 1][w]);
   int e_tot = ex.exk + norm_exp(um, 40);
   const float smax = G[P * P + P + 1];
   if (smax >= 1.17549435e-38f && smax < INFINITY) e_tot = min(e_tot, 111 - exp2_floor(smax));
   const float up = pow2i(e_tot - ex.exk);
-  // row i of B (K-major, no swizzle): K entries [U^_hi (PMAX) | U^_lo (PMAX) | U^_hi (PMAX, fp32 rows)]
-  uint32_t hi[PMAX / 2], lo[PMAX / 2];
+  // row i of B (K-major, no swizzle): K entries [U^_hi (PMAX) | U^_lo (PMAX) | U^_hi (PMAX, fp32 rows)];
+  // this thread writes entries sb .. sb + H2 - 1 of each segment
+  uint32_t hi[H2 / 2], lo[H2 / 2];
 #pragma unroll
-  for (int e = 0; e < PMAX / 2; ++e) {
+  for (int e = 0; e < H2 / 2; ++e) {
     const float2 a = __fmul2_rn(make_float2(u[2 * e], u[2 * e + 1]), make_float2(up, up));
     const __half2 h = __float22half2_rn(a);
     const float2 hf = __half22float2(h);
@@ -439,45 +467,47 @@ __device__ __forceinline__ void residual_update(const PoolDev& p, TcSmem<BF16, R
     lo[e] = h2u(__float22half2_rn(make_float2(a.x - hf.x, a.y - hf.y)));
   }
   uint8_t* row = sm.bu[t] + (i >> 3) * 256 + (i & 7) * 16;
-#pragma unroll
-  for (int c = 0; c < PMAX / 8; ++c) {
-    const int k0 = 8 * c, k1 = PMAX + 8 * c, k2 = 2 * PMAX + 8 * c;
-    *reinterpret_cast<uint4*>(row + (k0 >> 4) * 4096 + ((k0 >> 3) & 1) * 128) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-    *reinterpret_cast<uint4*>(row + (k1 >> 4) * 4096 + ((k1 >> 3) & 1) * 128) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-    if (C::NSEG == 3)
-      *reinterpret_cast<uint4*>(row + (k2 >> 4) * 4096 + ((k2 >> 3) & 1) * 128) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+  auto put = [&](int kk, const uint32_t (&w)[H2 / 2]) {
+    uint8_t* a = row + (kk >> 4) * 4096 + ((kk >> 3) & 1) * 128 + (kk & 7) * 2;
+    if constexpr (H2 == 4) *reinterpret_cast<uint2*>(a) = make_uint2(w[0], w[1]);
+    else *reinterpret_cast<uint4*>(a) = make_uint4(w[0], w[1], w[2], w[3]);
+  };
+  put(sb, hi);
+  put(PMAX + sb, lo);
+  if (C::NSEG == 3) put(2 * PMAX + sb, hi);
+  // epilogue factors, one tile position per thread of the first 128
+  if (ct < 128) {
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + code_bytes(C::D, C::D, bits));
+    const int j = bits == 4 ? chan_of<4>(ct) : ct;
+    sm.fj[m][ct] = gam[n - 1] * __half2float(__ushort_as_half(sc[j])) * pow2i(e_tot);
   }
-  // epilogue factors, one tile position per thread
-  const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + code_bytes(C::D, C::D, bits));
-  const int j = bits == 4 ? chan_of<4>(ct) : ct;
-  sm.fj[m][ct] = gam[n - 1] * __half2float(__ushort_as_half(sc[j])) * pow2i(e_tot);
   if (ct == 0) sm.meta_e[m] = e_tot;
 }
 
 template <bool BF16, bool R8, int PMAX>
 __device__ void converter_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uint32_t tm, int warp, int lane) {
   using C = TcCfg<BF16, R8, PMAX>;
-  const int cw = warp - C::CONV0, ct = 32 * cw + lane;
+  const int cw = warp - C::CONV0, ct = 32 * cw + lane;   // ct < NCT
   // Every wait is followed by a vote at the converters' named barrier, so that
   // the four warps leave together and none is left waiting in a barrier.
   for (int k = 0;; ++k) {
     const int s = k % C::NST, t = k & 1, m = k & 3;
     bool ok = bounded_wait(&sm.stage_full[s], (uint32_t)((k / C::NST) & 1), p, &sm.abort);
     const int head = ok ? sm.stage_head[s] : -1;
-    if (tc::named_sync_any(6, 128, !ok)) return;
+    if (tc::named_sync_any(6, C::NCT, !ok)) return;
     const uint8_t* st = sm.stage[s];
     const int bits = head >= 0 ? p.bits[head % p.H] : 4;
     // the tile and X's keys of buffer t were last read by the products of the
     // head two back, whose completion the previous R step waited for
     if (head >= 0) {
-      if (bits == 4) convert_codes<4>(st, sm.tile[t], cw, lane);
-      else convert_codes<8>(st, sm.tile[t], cw, lane);
+      if (bits == 4) convert_codes<4, 128 / C::NCONV>(st, sm.tile[t], cw, lane);
+      else convert_codes<8, 128 / C::NCONV>(st, sm.tile[t], cw, lane);
     }
     // the update of the head two back read this buffer's update keys; its
     // completion also means the epilogue of the head four back, which used
     // this ring slot, has read it
     if (k >= 2) ok = bounded_wait(&sm.acc_full[t], (uint32_t)(((k - 2) >> 1) & 1), p, &sm.abort);
-    if (tc::named_sync_any(6, 128, !ok)) return;
+    if (tc::named_sync_any(6, C::NCT, !ok)) return;
     if (head >= 0) {
       const int n = sm.stage_n[s];
       const KeyExp ex = key_exponents(reinterpret_cast<const float*>(st + C::REC + C::KVB), p.P);
@@ -493,7 +523,7 @@ __device__ void converter_role(const PoolDev& p, TcSmem<BF16, R8, PMAX>& sm, uin
     if (k >= 1) {   // R and U^ of the previous head, whose X has had this head's conversion to land
       const int sp = (k - 1) % C::NST, tp = t ^ 1;
       ok = bounded_wait(&sm.x_full[tp], (uint32_t)(((k - 1) >> 1) & 1), p, &sm.abort);
-      if (tc::named_sync_any(6, 128, !ok)) return;
+      if (tc::named_sync_any(6, C::NCT, !ok)) return;
       tc::fence_after_sync();
       const int hp = sm.stage_head[sp];
       residual_update<BF16, R8, PMAX>(p, sm, sm.stage[sp], p.bits[hp % p.H], tp, sm.stage_n[sp], tm, k - 1, ct,
@@ -537,6 +567,7 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
                                               uint32_t tm, int t, int m, int head, int we, int lane) {
   using C = TcCfg<BF16, R8, PMAX>;
   const int qd = we & 3, g = lane >> 2, q = lane & 3;
+  const int cb = (we - C::EPI0) >> 2;   // value-channel half of this warp (two warps per quadrant)
   const int e_tot = sm.meta_e[m];
   const float down = pow2i(-e_tot);
   float f[2][2];
@@ -545,7 +576,7 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
 #pragma unroll
     for (int h = 0; h < 2; ++h) f[blk][h] = sm.fj[m][32 * qd + 16 * blk + g + 8 * h];
   // S'^T of block blk, column half cb: v[4 c + 2 h + z] = rows 64 cb + 8 c + 2 q + z of lane g + 8 h
-  auto load = [&](int blk, int cb, float (&v)[32]) {
+  auto load = [&](int blk, float (&v)[32]) {
     uint32_t cr[32], ur[32];
     const uint32_t a = tm + ((uint32_t)(32 * qd + 16 * blk) << 16) + 256u * t + 64u * cb;
     tc::ld_16x256b_x8(a, cr);
@@ -563,19 +594,18 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
       }
   };
 
-  // pass 1: column maxima, 32 values per key channel here, then the other three lanes of the quad
+  // pass 1: column maxima, 16 values per key channel here, then the other
+  // three lanes of the quad, then the other value-channel half
   float mx[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-  for (int blk = 0; blk < 2; ++blk)
+  for (int blk = 0; blk < 2; ++blk) {
+    float v[32];
+    load(blk, v);
 #pragma unroll
-    for (int cb = 0; cb < 2; ++cb) {
-      float v[32];
-      load(blk, cb, v);
+    for (int c = 0; c < 8; ++c)
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) mx[blk][h] = max3_nan(mx[blk][h], fabsf(v[4 * c + 2 * h]), fabsf(v[4 * c + 2 * h + 1]));
-    }
+      for (int h = 0; h < 2; ++h) mx[blk][h] = max3_nan(mx[blk][h], fabsf(v[4 * c + 2 * h]), fabsf(v[4 * c + 2 * h + 1]));
+  }
 #pragma unroll
   for (int blk = 0; blk < 2; ++blk)
 #pragma unroll
@@ -583,6 +613,17 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
       mx[blk][h] = max_nan(mx[blk][h], __shfl_xor_sync(FULL, mx[blk][h], 1));
       mx[blk][h] = max_nan(mx[blk][h], __shfl_xor_sync(FULL, mx[blk][h], 2));
     }
+  if (q == 0) {
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) sm.emax[cb][32 * qd + 16 * blk + g + 8 * h] = mx[blk][h];
+  }
+  tc::named_sync(7 + qd, 64);   // the two warps of this quadrant
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) mx[blk][h] = max_nan(mx[blk][h], sm.emax[cb ^ 1][32 * qd + 16 * blk + g + 8 * h]);
 
   // scale of the column (blk, h) = (q >> 1, q & 1), then shared across the quad
   const int qmax = BITS == 4 ? 7 : 127;
@@ -596,7 +637,7 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
     sf = gs.sf;
     qf = gs.sf > 0.f ? __frcp_rn(gs.sf) * down : 0.f;
     bad = !fast_encode_ok(amax, gs, qmax) || !(qf < INFINITY);
-    reinterpret_cast<uint16_t*>(stg + 16384)[chan_of<BITS>(pos)] = gs.bits;
+    if (cb == 0) reinterpret_cast<uint16_t*>(stg + 16384)[chan_of<BITS>(pos)] = gs.bits;
   }
   const bool slow = __any_sync(FULL, bad);
   float qv[2][2];
@@ -615,13 +656,12 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
     };
     if (BITS == 4) {
       const uint32_t base = stg_a + 64 * r8 + ((qd ^ ((r8 >> 1) & 3)) << 4) + 512 * mq;
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
+      {
         uint32_t rb[2][8];   // [blk][c]: bytes 0 and 2 are the row pairs' code bytes
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           float v[32];
-          load(blk, cb, v);
+          load(blk, v);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             rb[blk][c] = (pair(v, blk, c, 0) & 0x000F000Fu) | ((pair(v, blk, c, 1) << 4) & ~0x000F000Fu);
@@ -636,10 +676,9 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
         const uint32_t base = stg_a + 128 * r8 + (((2 * qd + blk) ^ r8) << 4) + 1024 * mq;
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
+        {
           float v[32];
-          load(blk, cb, v);
+          load(blk, v);
           uint32_t w[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) w[c] = prmt(pair(v, blk, c, 0), pair(v, blk, c, 1), 0x6420u);
@@ -655,7 +694,7 @@ __device__ __forceinline__ void epilogue_head(const PoolDev& p, const CommitMaps
   tc::fence_before_sync();
   tc::mbar_arrive(&sm.tmem_empty[t]);
   fence_proxy_async_smem();
-  tc::named_sync(5, 128);
+  tc::named_sync(5, C::NET);
   if (we == C::EPI0 && lane == 0) {
     const int hh = head % p.H, b = head / p.H;
     const size_t off = (size_t)b * p.slot_stride + p.rec_off[hh];
@@ -677,7 +716,7 @@ __device__ void epilogue_role(const PoolDev& p, const CommitMaps& maps, TcSmem<B
     bool ok = bounded_wait(&sm.acc_full[t], (uint32_t)((k >> 1) & 1), p, &sm.abort);
     // the converters' per-head values (factors, exponent) are read directly after their arrival
     if (ok && sm.meta_head[m] >= 0) ok = bounded_wait(&sm.bupd_full[t], (uint32_t)((k >> 1) & 1), p, &sm.abort);
-    if (tc::named_sync_any(5, 128, !ok)) break;
+    if (tc::named_sync_any(5, TcCfg<BF16, R8, PMAX>::NET, !ok)) break;
     tc::fence_after_sync();
     const int head = sm.meta_head[m];
     if (head < 0) break;
@@ -699,14 +738,14 @@ __global__ void __launch_bounds__(TcCfg<BF16, R8, PMAX>::THREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&sm.stage_full[s], 1);
-      mbar_init(&sm.stage_empty[s], 128);
+      mbar_init(&sm.stage_empty[s], C::NCT);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&sm.tile_full[t], 128);
+      mbar_init(&sm.tile_full[t], C::NCT);
       mbar_init(&sm.x_full[t], 1);
-      mbar_init(&sm.bupd_full[t], 128);
+      mbar_init(&sm.bupd_full[t], C::NCT);
       mbar_init(&sm.acc_full[t], 1);
-      mbar_init(&sm.tmem_empty[t], 128);
+      mbar_init(&sm.tmem_empty[t], C::NET);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
