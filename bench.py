@@ -41,6 +41,8 @@ def parse_args():
     ap.add_argument("--workload", default="concurrency_stress")
     ap.add_argument("--period", type=int, default=None, help="override P")
     ap.add_argument("--axis", choices=["col", "row"], default=None, help="override the scale axis")
+    ap.add_argument("--commit-engine", choices=["tcgen05", "mma"], default="tcgen05",
+                    help="period-commit kernel (tcgen05 falls back to mma for shapes it is not built for)")
     ap.add_argument("--prefill-tokens", type=int, default=64,
                     help="tokens of the chunked fp32 prefill measured after the decode (0: skip)")
     ap.add_argument("--commit-threshold", default=None,
@@ -72,6 +74,17 @@ def parse_args():
 
 # ----------------------------------------------------------------------------- helpers
 
+def tensor_peak():
+    """Dense bf16/f16 tensor peak in TFLOP/s for a kernel timed inside a long
+    step (the sustained figure of MEASURED_PEAKS.json; fallback 1400)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1400.0, "fallback"
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -82,15 +95,16 @@ def measured_peaks():
         return HBM_FALLBACK_GBS, "fallback"
 
 
-KERNEL_SOURCES = {"decode_step": "decode_kernels.cu", "commit": "commit_kernels.cu"}
+KERNEL_SOURCES = {"decode_step": "decode_kernels.cu", "commit": "commit_tc_kernels.cu"}
+COMMIT_SOURCES = {"tcgen05": "commit_tc_kernels.cu", "mma": "commit_kernels.cu"}
 
 
-def kernel_source_digest(kernel: str) -> str:
+def kernel_source_digest(kernel: str, source: str = None) -> str:
     """sha256 (16 hex digits) of a kernel's source file and every csrc header
     it includes, directly or not: what a DRAM-traffic record depends on."""
     import re
     csrc = os.path.join(ROOT, "bit_recurrent_state_pace_b200", "csrc")
-    todo, seen = [KERNEL_SOURCES[kernel]], []
+    todo, seen = [source or KERNEL_SOURCES[kernel]], []
     while todo:
         fn = todo.pop()
         if fn in seen or not os.path.exists(os.path.join(csrc, fn)):
@@ -371,6 +385,12 @@ def run_pace(args, rank: int, world: int):
         bits = pace.pace_select_head_bits(rates.cpu().tolist(), sum(1 for b in bits if b == 8))
         del gates
     pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, P, bits, axis=w.axis, io=w.io_dtype, device=dev)
+    engine = args.commit_engine
+    try:
+        pool.set_commit_engine(pace.PACE_COMMIT_TCGEN05 if engine == "tcgen05" else pace.PACE_COMMIT_MMA)
+    except pace.PaceError:
+        engine = "mma"
+        pool.set_commit_engine(pace.PACE_COMMIT_MMA)
     pool.load(S)
     S_bf16 = None if args.no_compare else S.to(torch.bfloat16).view(torch.int16)
     del S
@@ -428,7 +448,8 @@ def run_pace(args, rank: int, world: int):
     hbm, peak_kind = measured_peaks()
     dec_gbs = dec_avg_bytes / (dec_avg_ms * 1e-3) / 1e9
     com_gbs = com_bytes / (com_avg_ms * 1e-3) / 1e9
-    digest = {kern: kernel_source_digest(kern) for kern in KERNEL_SOURCES}
+    digest = {"decode_step": kernel_source_digest("decode_step"),
+              "commit": kernel_source_digest("commit", COMMIT_SOURCES[engine])}
     dominant = "decode_step" if dec_avg_ms * P >= com_avg_ms else "commit"
     ach = dec_gbs if dominant == "decode_step" else com_gbs
     traffic = ncu_traffic(dominant, digest[dominant])
@@ -528,9 +549,16 @@ def run_pace(args, rank: int, world: int):
         esz = 2 if w.io_dtype == "bf16" else 4
         pbytes = (Tp * BH * ((2 * w.d_k + w.d_v + 2) * esz + 4 * w.d_v) + 2 * int(pool.state.numel()))
         from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+        # flops: per head-token S k, S q and the rank-one write, 2 d_k d_v each
+        pflops = 6.0 * w.d_k * w.d_v * BH * Tp
+        tpk, tpk_kind = tensor_peak()
+        ach_tf = pflops / (pms * 1e-3) / 1e12
         prefill = {"tokens": Tp, "value": aggregate_rate(BH * Tp, world, pms), "unit": "head-tokens/s",
                    "ms": pms, "alg_bytes": pbytes, "achieved_gbs": pbytes / (pms * 1e-3) / 1e9,
                    "frac_of_peak": pbytes / (pms * 1e-3) / 1e9 / measured_peaks()[0],
+                   "roofline_flops": {"bound": "tensor", "achieved": ach_tf, "peak": tpk, "unit": "TFLOP/s",
+                                      "frac": ach_tf / tpk, "flops_per_head_token": 6 * w.d_k * w.d_v,
+                                      "peak_source": f"{tpk_kind} bf16_tflops_sustained (f16 operands, same rate)"},
                    "status": pool.status()}
         del pin, po
 
@@ -564,6 +592,7 @@ def run_pace(args, rank: int, world: int):
                 "commit": {"avg_ms": com_avg_ms, "alg_bytes_per_launch": com_bytes,
                            "achieved_gbs": com_gbs, "frac_of_peak": com_gbs / hbm},
                 "source_digest": digest,
+                "commit_engine": engine,
             },
             "clocks": clocks,
             "e2e": e2e,

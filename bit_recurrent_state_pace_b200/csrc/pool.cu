@@ -188,6 +188,8 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
   }
   if (desc->d_k == 128 && desc->d_v == 128)
     p->maps_ok = pace::make_commit_maps(dv.state, L.state_bytes, &p->maps);
+  // the tensor-memory commit where it is built for the shape, else mma.sync
+  p->commit_engine = p->maps_ok && pace::commit_tc_supported(dv) ? PACE_COMMIT_TCGEN05 : PACE_COMMIT_MMA;
   cudaError_t e = cudaMemsetAsync(d_aux, 0, L.aux_bytes, as_stream(stream));
   if (e != cudaSuccess) {
     delete p;

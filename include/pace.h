@@ -204,12 +204,14 @@ pace_status pace_commit_period(pace_pool* pool, void* stream);
  * Which kernel applies the period commit (same results: both encode the
  * fp32 update of the page's chunked, high-precision period end, see
  * pace_commit_period; codes may differ only at exact rounding ties).
- *  PACE_COMMIT_MMA (default): warp-level tensor-core products (mma.sync)
- *    with the update and the encode in registers; every pool shape.
+ *  PACE_COMMIT_MMA: warp-level tensor-core products (mma.sync) with the
+ *    update and the encode in registers; every pool shape.
  *  PACE_COMMIT_TCGEN05: fifth-generation tensor cores with the update in
  *    tensor memory and the records written back by TMA stores; pools with
  *    d_k = d_v = 128 and column scales (fp32 io only with P <= 8), else
  *    PACE_ERR_UNSUPPORTED.
+ * A new pool starts with PACE_COMMIT_TCGEN05 where that engine is built for
+ * its shape, else PACE_COMMIT_MMA.
  * Host-only; applies to launches enqueued after the call.  Any other value
  * is PACE_ERR_INVALID_ARG.
  */

@@ -1,8 +1,8 @@
-"""The tensor-memory commit engine (PACE_COMMIT_TCGEN05) against the fp64
-oracle, teacher-forced per period as in test_gpu_decode: outputs within
-2e-3, committed codes equal up to +-1 at rounding ties (<= 0.1 %).  Pools of
-192 heads make every CTA of the persistent grid carry several heads through
-its pipeline.  Also: the two engines commit the same codes from the same
+"""Both commit engines (PACE_COMMIT_TCGEN05, the default where it is built
+for the shape, and PACE_COMMIT_MMA) against the fp64 oracle, teacher-forced
+per period as in test_gpu_decode: outputs within 2e-3, committed codes equal
+up to +-1 at rounding ties (<= 0.1 %).  Pools of 192 heads make every CTA of
+the persistent grid carry several heads through its pipeline.  Also: the two engines commit the same codes from the same
 buffered tokens, and shapes the engine is not built for are refused."""
 import numpy as np
 import pytest
@@ -20,6 +20,7 @@ def _pace():
     return pace
 
 
+@pytest.mark.parametrize("engine", ["tcgen05", "mma"])
 @pytest.mark.parametrize("name,over", [
     ("gdn_layer_4b", dict(B=6)),
     ("mixed_4_8", dict(B=6)),
@@ -28,10 +29,11 @@ def _pace():
     ("mixed_4_8", dict(B=3, P=8, io_dtype="f32")),
     ("gdn_layer_4b", dict(B=3, P=1)),
 ])
-def test_tcgen05_commit_against_oracle(name, over):
+def test_commit_engines_against_oracle(name, over, engine):
     pace = _pace()
     w = pace_synth.workload(name, **over)
-    worst, stats = _run_periods(w, periods=2, seed=3, warm_tokens=32, engine=pace.PACE_COMMIT_TCGEN05)
+    eng = pace.PACE_COMMIT_TCGEN05 if engine == "tcgen05" else pace.PACE_COMMIT_MMA
+    worst, stats = _run_periods(w, periods=2, seed=3, warm_tokens=32, engine=eng)
     assert worst <= pu.O_TOL
     print(name, over, "worst", worst, [s["codes_differing"] for s in stats])
 
@@ -44,6 +46,7 @@ def test_engines_commit_the_same_codes(P):
     S = pace_synth.random_state(w.B * w.H, w.d_v, w.d_k, seed=9, device="cuda").view(w.B, w.H, w.d_v, w.d_k)
     a = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype)
     b = pace.PacePool(w.B, w.H, w.d_k, w.d_v, w.P, bits, axis=w.axis, io=w.io_dtype)
+    a.set_commit_engine(pace.PACE_COMMIT_MMA)
     b.set_commit_engine(pace.PACE_COMMIT_TCGEN05)
     a.load(S)
     b.load(S)
