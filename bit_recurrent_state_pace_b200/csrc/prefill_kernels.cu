@@ -39,6 +39,7 @@ struct PCfg {
   static constexpr int NSEG = BF16 ? 2 : 3;         // update segments (K, K, K_lo)
   static constexpr int KU = (NSEG * CH + 15) / 16;  // update k16 steps
   static constexpr int NKX = BF16 ? 2 : 4;          // K, Q (+ K_lo, Q_lo) operand tiles
+  static constexpr int MINB = D == 128 ? 2 : 1;     // CTAs (heads) in flight per SM
 };
 
 template <int D, bool BF16>
@@ -589,7 +590,7 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(PCfg<D, BF16>::THREADS, 1)
+__global__ void __launch_bounds__(PCfg<D, BF16>::THREADS, PCfg<D, BF16>::MINB)
     prefill_kernel(PoolDev p, Span sp, int64_t T, const void* __restrict__ q,
                    const void* __restrict__ k, const void* __restrict__ v,
                    const void* __restrict__ alpha, const void* __restrict__ beta,
@@ -622,7 +623,7 @@ cudaError_t launch_t(const PoolDev& p, const Span& sp, int64_t T, const void* q,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  long blocks = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 1) * sms * (D == 128 ? 1 : D == 64 ? 2 : 4);
+  long blocks = (long)(sp.blocks_per_sm > 0 ? sp.blocks_per_sm : 1) * sms * (D == 128 ? PCfg<D, BF16>::MINB : D == 64 ? 2 : 4);
   if (blocks > heads) blocks = heads;
   prefill_kernel<D, BF16><<<(unsigned)blocks, PCfg<D, BF16>::THREADS, smem, st>>>(p, sp, T, q, k, v,
                                                                                  alpha, beta, o);
