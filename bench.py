@@ -646,20 +646,23 @@ def run_period_sweep(args, pace, dev, mk):
                                io_code, None, BH, w0.d_k, w0.d_v)
     toks = [pace_synth.token_inputs(w0, t, seed=args.seed, device=dev) for t in range(T)]
 
-    # the unquantised trajectory from the encoded start
-    pool = pace.PacePool(w0.B, w0.H, w0.d_k, w0.d_v, 1, bits, axis=w0.axis, io=w0.io_dtype, device=dev)
-    pool.load(S)
-    S_ref = pool.export().view(BH, w0.d_v, w0.d_k).contiguous()
-    del pool
+    # the unquantised trajectory from the encoded start, for each scale axis run
     o = torch.empty(w0.B, w0.H, w0.d_v, dtype=torch.float32, device=dev)
-    ref = {}
-    for t in range(T):
-        x = toks[t]
-        pace.pace_gdn_step_f32(S_ref, x["q"], x["k"], x["v"], x["alpha"], x["beta"], io_code, o,
-                               BH, w0.d_k, w0.d_v)
-        if t + 1 in horizons:
-            ref[t + 1] = o.clone()
-    del S_ref
+    refs = {}
+    for axis in ("col", "row"):
+        pool = pace.PacePool(w0.B, w0.H, w0.d_k, w0.d_v, 1, bits, axis=axis, io=w0.io_dtype, device=dev)
+        pool.load(S)
+        S_ref = pool.export().view(BH, w0.d_v, w0.d_k).contiguous()
+        del pool
+        ref = {}
+        for t in range(T):
+            x = toks[t]
+            pace.pace_gdn_step_f32(S_ref, x["q"], x["k"], x["v"], x["alpha"], x["beta"], io_code, o,
+                                   BH, w0.d_k, w0.d_v)
+            if t + 1 in horizons:
+                ref[t + 1] = o.clone()
+        refs[axis] = ref
+        del S_ref
     hbm = measured_peaks()[0]
 
     def drift(out, r):
@@ -669,8 +672,12 @@ def run_period_sweep(args, pace, dev, mk):
         return {"mean": float(e.mean()), "max": float(e.max())}
 
     rows = []
-    for P in pace_synth.PERIOD_SWEEP:
-        w = w0.replace(P=P)
+    # the workload's column scales at every P, and row scales (one scale per
+    # value channel, the group that holds the outlier channels) at P = 8
+    runs = [(P, "col") for P in pace_synth.PERIOD_SWEEP] + [(8, "row")]
+    for P, axis in runs:
+        w = w0.replace(P=P, axis=axis)
+        ref = refs[axis]
         pool = pace.PacePool(w.B, w.H, w.d_k, w.d_v, P, bits, axis=w.axis, io=w.io_dtype, device=dev)
         pool.load(S)
         dev_ev = [(mk(), mk()) for _ in range(T)]
@@ -702,7 +709,7 @@ def run_period_sweep(args, pace, dev, mk):
         dec_gbs = sum(dec_bytes) / (sum(dec_ms) * 1e-3) / 1e9
         com_gbs = com_bytes * len(com_ms) / (sum(com_ms) * 1e-3) / 1e9 if com_ms else None
         rows.append({
-            "P": P, "tokens": T,
+            "P": P, "axis": axis, "commit_engine": "tcgen05" if axis == "col" else "mma", "tokens": T,
             "value": BH * T / (kern_ms * 1e-3), "unit": "head-tokens/s",
             "ms_per_token": kern_ms / T,
             "wall_ms": a.elapsed_time(b),
@@ -714,15 +721,17 @@ def run_period_sweep(args, pace, dev, mk):
             "device_status": status,
         })
         del pool, got
-    del toks, S, ref
+    del toks, S, refs
     torch.cuda.synchronize()
     return {
         "workload": f"period_sweep: B={w0.B} H={w0.H} d_k={w0.d_k} d_v={w0.d_v}, all INT4, "
-                    f"{w0.axis} scales, {w0.io_dtype} io, {w0.warmup}-token fp32 warm-up, {T} decode tokens",
+                    f"{w0.axis} scales at P in {list(pace_synth.PERIOD_SWEEP)} and row scales at P = 8, "
+                    f"{w0.io_dtype} io, {w0.warmup}-token fp32 warm-up, {T} decode tokens",
         "state_bytes": state_bytes_of(w0, bits),
         "l2": "state pool 138 MB, near the 126 MB L2: no flush; part of the traffic is served from L2",
         "drift_metric": "per head ||o - o_fp32||_inf / ||o_fp32||_inf at token t (mean, max over heads); "
-                        "o_fp32 from pace_gdn_step_f32 started at the encoded warm state, dequantised",
+                        "o_fp32 from pace_gdn_step_f32 started at the encoded warm state (same scale axis), "
+                        "dequantised",
         "time": "sum of per-launch CUDA-event durations (value); wall_ms includes the output copies "
                 "taken at the horizons",
         "rows": rows,

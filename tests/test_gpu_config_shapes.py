@@ -1,9 +1,10 @@
 """The gated-delta layer, mixed 4/8-bit and period-sweep workloads at their
 stated shapes, run for their stated numbers of decode steps.
 
-* gdn_layer_4b: B = 64 x H = 32, d = 128, P = 8, all INT4, 256 decode steps;
+* gdn_layer_4b: B = 64 x H = 32, d = 128, P = 8, all INT4, 256 decode steps,
+  with column scales and with row scales;
 * mixed_4_8: B = 256 x H = 32, P = 8, 8 of 32 heads INT8 (the long-memory
-  heads), 512 decode steps;
+  heads), 512 decode steps, with column scales and with row scales;
 * period_sweep: B = 512 x H = 32, all INT4, 1024 decode steps for each
   P in {1, 2, 4, 8, 16} (P = 1 rounds after every token).
 
@@ -101,19 +102,21 @@ def _run(w, bits, heads, S_warm, state):
     return worst
 
 
-def test_gdn_layer_4b_full_shape():
-    w = pace_synth.workload("gdn_layer_4b")
+@pytest.mark.parametrize("axis", ["col", "row"])
+def test_gdn_layer_4b_full_shape(axis):
+    w = pace_synth.workload("gdn_layer_4b", axis=axis)
     assert (w.B, w.H, w.P, w.steps, w.warmup) == (64, 32, 8, 256, 512)
     bits = pace_synth.head_bits(w, SEED)
     heads = _sample_heads(w, bits, n_random=28)
     S = _warm_pool_state(_pace(), w)
     state = pu.oracle_warm_state(w, heads, [bits[h] for _, h in heads], seed=SEED, device="cuda")
     worst = _run(w, bits, heads, S, state)
-    print(f"gdn_layer_4b: {len(heads)} heads x {w.steps} tokens, worst relative error {worst:.3e}")
+    print(f"gdn_layer_4b ({axis}): {len(heads)} heads x {w.steps} tokens, worst relative error {worst:.3e}")
 
 
-def test_mixed_4_8_full_shape():
-    w = pace_synth.workload("mixed_4_8")
+@pytest.mark.parametrize("axis", ["col", "row"])
+def test_mixed_4_8_full_shape(axis):
+    w = pace_synth.workload("mixed_4_8", axis=axis)
     bits = pace_synth.head_bits(w, SEED)
     assert (w.B, w.H, w.steps) == (256, 32, 512) and sum(b == 8 for b in bits) == 8
     heads = _sample_heads(w, bits, n_random=20, n_int8=12)
@@ -121,7 +124,7 @@ def test_mixed_4_8_full_shape():
     S = _warm_pool_state(_pace(), w)
     state = pu.oracle_warm_state(w, heads, [bits[h] for _, h in heads], seed=SEED, device="cuda")
     worst = _run(w, bits, heads, S, state)
-    print(f"mixed_4_8: {len(heads)} heads x {w.steps} tokens, worst relative error {worst:.3e}")
+    print(f"mixed_4_8 ({axis}): {len(heads)} heads x {w.steps} tokens, worst relative error {worst:.3e}")
 
 
 @pytest.fixture(scope="module")
