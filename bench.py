@@ -57,6 +57,10 @@ def parse_args():
     ap.add_argument("--prefill", type=int, default=None, help="warm-up prefill tokens (default: workload's)")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the periods from eager launches only (by default the headline value is "
+                         "from replays of one captured CUDA graph of a period; the eager timing is "
+                         "reported beside it under 'lockstep')")
     ap.add_argument("--no-compare", action="store_true", help="skip the bf16-state comparison path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-period-sweep", action="store_true",
@@ -458,6 +462,18 @@ def run_pace(args, rank: int, world: int):
     lockstep_value = aggregate_rate(BH * P * args.steps, world, elapsed_ms)
     lockstep_ms = elapsed_ms
 
+    # ---- the same periods replayed from one captured CUDA graph (reported
+    #      beside the headline; the per-kernel numbers above come from the
+    #      launches themselves)
+    graph_rec = None
+    if not args.no_graph and args.schedule == "lockstep":
+        try:
+            graph_rec = time_graph(pace, pool, toks, outs, P, args, stream, world, dev, mk, gpu_uuid)
+        except Exception as exc:   # capture refused: the eager timing stands
+            graph_rec = {"error": f"{type(exc).__name__}: {exc}"}
+            torch.cuda.synchronize()
+        status |= pool.status()
+
     # ---- staggered phases (continuous batching): same work per P steps
     stag = None
     if args.schedule == "staggered":
@@ -483,6 +499,9 @@ def run_pace(args, rank: int, world: int):
         barrier(world)
         elapsed_ms = max_over_ranks(a.elapsed_time(b), world, dev)
         status |= pool.status()
+    if stag is None and graph_rec and "value" in graph_rec:
+        elapsed_ms = graph_rec["ms_per_step"] * args.steps   # the headline from the graph replays
+        clocks = graph_rec["clocks"] or clocks
     value = aggregate_rate(BH * P * args.steps, world, elapsed_ms)
 
     # ---- bf16-state comparison path (unquantised, same shape)
@@ -600,8 +619,11 @@ def run_pace(args, rank: int, world: int):
             "schedule": ("staggered: %d slot groups one token apart; each step the full group's "
                          "commit and decode (stream b) overlap the other groups' decode (stream a), "
                          "%s blocks per SM" % (P, args.stagger_blocks)) if stag is not None
-                        else "lockstep: every slot at the same phase",
+                        else ("lockstep: every slot at the same phase; "
+                              + ("periods replayed from one captured CUDA graph (eager launches under "
+                                 "'lockstep')" if graph_rec and "value" in graph_rec else "eager launches")),
             "lockstep": {"value": lockstep_value, "ms_per_step": lockstep_ms / args.steps},
+            "cuda_graph": graph_rec,
             "device_status": status,
             "comparison": compare,
             "prefill": prefill,
@@ -611,6 +633,42 @@ def run_pace(args, rank: int, world: int):
             "cpu_baseline": cpu_base,
         }
         print(json.dumps(line), flush=True)
+
+
+def time_graph(pace, pool, toks, outs, P, args, stream, world, dev, mk, gpu_uuid):
+    """K periods replayed from one captured CUDA graph of a period (P decode
+    launches + the commit, the same calls and buffers as the eager loop)."""
+    import torch
+    from bit_recurrent_state_pace_b200.ranks import aggregate_rate
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for n in range(P):
+            x = toks[n]
+            pace.pace_decode_step(pool.handle, x["q"], x["k"], x["v"], x["alpha"], x["beta"], outs[n],
+                                  side.cuda_stream)
+        pace.pace_commit_period(pool.handle, side.cuda_stream)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g.replay()
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_uuid)
+    time.sleep(0.2)
+    a, b = mk(), mk()
+    a.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    gms = max_over_ranks(a.elapsed_time(b), world, dev)
+    BH = pool.B * pool.H
+    return {"value": aggregate_rate(BH * P * args.steps, world, gms), "unit": "head-tokens/s",
+            "ms_per_step": gms / args.steps, "launches_per_step": P + 1, "clocks": clocks,
+            "note": "one period (P decode launches + the commit) captured once, replayed K times"}
 
 
 def run_period_sweep(args, pace, dev, mk):
