@@ -103,9 +103,19 @@ KERNEL_SOURCES = {"decode_step": "decode_kernels.cu", "commit": "commit_tc_kerne
 COMMIT_SOURCES = {"tcgen05": "commit_tc_kernels.cu", "mma": "commit_kernels.cu"}
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and with whitespace collapsed: edits to
+    comments do not change what a traffic record was measured on."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_digest(kernel: str, source: str = None) -> str:
     """sha256 (16 hex digits) of a kernel's source file and every csrc header
-    it includes, directly or not: what a DRAM-traffic record depends on."""
+    it includes, directly or not, comments left out: what a DRAM-traffic
+    record depends on."""
     import re
     csrc = os.path.join(ROOT, "bit_recurrent_state_pace_b200", "csrc")
     todo, seen = [source or KERNEL_SOURCES[kernel]], []
@@ -118,8 +128,8 @@ def kernel_source_digest(kernel: str, source: str = None) -> str:
             todo += re.findall(r'^#include "([^"/]+)"', f.read(), flags=re.M)
     h = hashlib.sha256()
     for fn in sorted(seen):
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + f.read())
+        with open(os.path.join(csrc, fn)) as f:
+            h.update(fn.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

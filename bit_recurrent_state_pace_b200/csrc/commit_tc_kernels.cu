@@ -11,26 +11,30 @@
 // with W[s][s'] = gamma_{n/s} T[s][s'] beta_s', T = (I + A)^{-1}, left in the
 // head's factor block by the decode step that filled the buffer.
 //
-// Design (one CTA per SM, warp-specialised, two heads in flight):
-//  * producer warp: finds the heads due for a commit and stages each one's
-//    record, buffered rows and factor block in shared memory by 1-D bulk
-//    copies (no multicast), several heads ahead;
-//  * converter warps (4): turn the codes into one exact f16 tile, [i][j] with
-//    128-byte swizzling, that serves two MMAs: read K-major it is the A of
-//    X = C (diag(s) K^T) and read MN-major it is the A of C^T = C^T I, a
-//    transpose by block-identity products (N = 16 per block).  They also
-//    build the scaled keys of both products, and, once X is in TMEM, compute
-//    R and U^ for their TMEM lane (value channel i) and write U^ as the B of
-//    the update;
+// Design (one CTA of 18 warps per SM, warp-specialised, two heads in flight;
+// each CTA takes its 4-bit heads before its 8-bit heads):
+//  * producer warp: finds the heads due for a commit (one ballot over 32 fill
+//    counters per global round trip) and stages each one's record, buffered
+//    rows and factor block in shared memory by 1-D bulk copies (no
+//    multicast), several heads ahead;
+//  * converter warps (8, two per TMEM lane quadrant): turn the codes into one
+//    exact f16 tile, [i][j] with 128-byte swizzling, that serves two MMAs:
+//    read K-major it is the A of X = C (diag(s) K^T) and read MN-major it is
+//    the A of C^T = C^T I, a transpose by block-identity products (N = 16 per
+//    block).  They also build the scaled keys of both products, and, once X
+//    is in TMEM, compute R and U^ for their TMEM lane (value channel i), the
+//    two warps of a quadrant each for half of the tokens, and write U^ as the
+//    B of the update;
 //  * MMA warp: issues X and the transpose into TMEM (f32), then the update
 //    U^T = K^T U^ (key channels on TMEM lanes, value channels on columns),
 //    hi/lo f16 splits, fp32 accumulation;
-//  * epilogue warps (8, two per TMEM lane quadrant): S^T = gamma_n s_j C^T +
-//    U^T with one fma per element, per-column absmax thread-local plus two
-//    shuffles, FP16 scales, round-half-even codes by the f16 magic number,
-//    bytes transposed into a swizzled staging area by stmatrix, and the
-//    record written back by one tensor store (codes) and one bulk store
-//    (scales).
+//  * epilogue warps (8, two per TMEM lane quadrant, one per half of the value
+//    channels): S^T = gamma_n s_j C^T + U^T with one fma per element,
+//    per-column absmax thread-local plus two shuffles and one exchange
+//    between the quadrant's two warps, FP16 scales, round-half-even codes by
+//    the f16 magic number, bytes transposed into a swizzled staging area by
+//    stmatrix, and the record written back by one tensor store (codes) and
+//    one bulk store (scales).
 // Every wait is bounded; a wait that gives up sets PACE_FLAG_TIMEOUT and the
 // CTA drains its tensor work, frees TMEM and returns.
 #include <type_traits>
