@@ -44,12 +44,13 @@ constexpr int kWarpsPerBlock = 8;
 constexpr int kThreads = kWarpsPerBlock * 32;
 constexpr unsigned FULL = 0xffffffffu;
 
-// ADAPT (commit threshold set): two more right-hand sides, a^ and b^ (digit
-// rows 4..6 and 8..10), for the accumulated-update norm.
+// ADAPT (commit threshold set): two more right-hand sides, a^ and b^, as two
+// digits each (rows 3..4 and 5..6; row 7 zeros), for the accumulated-update
+// norm: all three fit one n8 product.
 template <int D, bool ADAPT>
 struct alignas(16) WarpScratch {
-  static constexpr int NDIG = ADAPT ? 11 : 4;
-  uint8_t dig[NDIG][D];            // digits 0..2 of q^ (row 3 = zeros), then of a^, b^
+  static constexpr int NDIG = ADAPT ? 8 : 4;
+  uint8_t dig[NDIG][D];            // digits 0..2 of q^, then (ADAPT) 0..1 of a^ and b^; last row zeros
   float y[D];                      // S~0 q^ by row, before the row scale
   float ya[ADAPT ? D : 1];         // S~0 a^
   float yb[ADAPT ? D : 1];         // S~0 b^
@@ -115,6 +116,64 @@ template <int BITS>
 __device__ __forceinline__ void offset_corr(const int (&dsum)[3], int (&corr)[3]) {
 #pragma unroll
   for (int d = 0; d < 3; ++d) {
+    int v2 = dsum[d];
+    if (BITS == 4) {
+#pragma unroll
+      for (int off = 16; off; off >>= 1) v2 += __shfl_xor_sync(FULL, v2, off);
+    }
+    corr[d] = BITS == 4 ? 8 * v2 : 0;
+  }
+}
+
+// The same split with two digits (14-bit fixed point: x 2^e = d0 + 256 d1,
+// |x 2^e| < 2^14), for the norm-tracking right-hand sides, where 14 bits are
+// ample: they only decide when to commit, not what is committed.
+template <int D, int EPL, int BITS>
+__device__ __forceinline__ float rhs_digits2(const float (&x)[EPL], uint8_t (*dig)[D], int lane,
+                                             int (&dsum)[2]) {
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+  int ex = 0;
+  if (m > 0.f && m < INFINITY) ex = max(-120, min(120, 13 - ilogbf(m)));
+  const float up = ldexpf(1.f, ex);
+  dsum[0] = dsum[1] = 0;
+  uint32_t dw[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int Q = __float2int_rn(x[e] * up);
+    const int d0 = (int)(int8_t)(Q & 0xff);
+    const int d1 = (Q - d0) >> 8;
+    dsum[0] += d0; dsum[1] += d1;
+    dw[0] |= (uint32_t)(d0 & 0xff) << (8 * e);
+    dw[1] |= (uint32_t)(d1 & 0xff) << (8 * e);
+  }
+  if (BITS == 8) {
+#pragma unroll
+    for (int d = 0; d < 2; ++d) {
+      uint8_t* dst = &dig[d][EPL * lane];
+      if (EPL == 4) *reinterpret_cast<uint32_t*>(dst) = dw[d];
+      else if (EPL == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)dw[d];
+      else *dst = (uint8_t)dw[d];
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int j = EPL * lane + e, o = j & 7;
+      const int at = (j & ~7) + ((o & 1) ? 4 + (o >> 1) : (o >> 1));
+#pragma unroll
+      for (int d = 0; d < 2; ++d) dig[d][at] = (uint8_t)(dw[d] >> (8 * e));
+    }
+  }
+  return ldexpf(1.f, -ex);
+}
+
+template <int BITS>
+__device__ __forceinline__ void offset_corr2(const int (&dsum)[2], int (&corr)[2]) {
+#pragma unroll
+  for (int d = 0; d < 2; ++d) {
     int v2 = dsum[d];
     if (BITS == 4) {
 #pragma unroll
@@ -393,7 +452,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
   const float down = rhs_digits<D, EPL, BITS>(bv, &scr.dig[0], lane, dsum);
   offset_corr<BITS>(dsum, corr);
   float down_a = 0.f, down_b = 0.f;
-  int corr_a[3] = {0, 0, 0}, corr_b[3] = {0, 0, 0};
+  int corr_a[2] = {0, 0}, corr_b[2] = {0, 0};
   if constexpr (ADAPT) {
     float av[EPL], bw[EPL];
 #pragma unroll
@@ -402,22 +461,28 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
       av[e] = col ? ah * sc[e] : ah;
       bw[e] = col ? bh[e] * sc[e] : bh[e];
     }
-    down_a = rhs_digits<D, EPL, BITS>(av, &scr.dig[4], lane, dsum);
-    offset_corr<BITS>(dsum, corr_a);
-    down_b = rhs_digits<D, EPL, BITS>(bw, &scr.dig[8], lane, dsum);
-    offset_corr<BITS>(dsum, corr_b);
+    int ds2[2];
+    down_a = rhs_digits2<D, EPL, BITS>(av, &scr.dig[3], lane, ds2);
+    offset_corr2<BITS>(ds2, corr_a);
+    down_b = rhs_digits2<D, EPL, BITS>(bw, &scr.dig[5], lane, ds2);
+    offset_corr2<BITS>(ds2, corr_b);
   }
   __syncwarp();
   constexpr int NC = D / 32;           // k32 chunks
-  // columns 0..2: q^ digits; ADAPT: 4..6 a^ digits (second product: 0..2 b^)
-  uint32_t bfr[NC][2], bfr2[NC][2];
-  load_bfrag<D, BITS>(&scr.dig[g < 3 || (ADAPT && g >= 4 && g < 7) ? g : 3][0], t, bfr);
-  if constexpr (ADAPT) load_bfrag<D, BITS>(&scr.dig[g < 3 ? 8 + g : 3][0], t, bfr2);
+  // columns 0..2: q^ digits (3..7 zero); ADAPT: 3..4 a^ digits, 5..6 b^ digits, 7 zero
+  uint32_t bfr[NC][2];
+  if constexpr (ADAPT) load_bfrag<D, BITS>(&scr.dig[g][0], t, bfr);
+  else load_bfrag<D, BITS>(&scr.dig[g < 3 ? g : 3][0], t, bfr);
   // accumulator columns 2t, 2t+1 of lane t: (d0, d1) for even t, (d2, -) for odd t
-  const int cA = t == 0 ? corr[0] : t == 1 ? corr[2] : t == 2 ? corr_a[0] : corr_a[2];
-  const int cB = t == 0 ? corr[1] : t == 2 ? corr_a[1] : 0;
-  const int cA2 = t == 0 ? corr_b[0] : t == 1 ? corr_b[2] : 0;
-  const int cB2 = t == 0 ? corr_b[1] : 0;
+  const int cA = t == 0 ? corr[0] : t == 1 ? corr[2] : 0;
+  const int cB = t == 0 ? corr[1] : 0;
+  // ADAPT: the weight (256^digit) and offset correction of lane t's two
+  // columns: t = 0: q^ d0, d1; t = 1: q^ d2, a^ d0; t = 2: a^ d1, b^ d0;
+  // t = 3: b^ d1, zero.  Lane t then adds the first column of lane t + 1 to
+  // its own and holds q^ (t = 0), a^ (t = 1) or b^ (t = 2).
+  const float aw0 = t == 1 ? 65536.f : t == 0 ? 1.f : 256.f, aw1 = t == 0 ? 256.f : t == 3 ? 0.f : 1.f;
+  const int ak0 = t == 0 ? corr[0] : t == 1 ? corr[2] : t == 2 ? corr_a[1] : corr_b[1];
+  const int ak1 = t == 0 ? corr[1] : t == 1 ? corr_a[0] : t == 2 ? corr_b[0] : 0;
 
   // 9. y = S~0 (codes) x b on the int8 tensor cores (exact int32), 16 rows at a time
   // (unrolled by the prefetch depth only: a smaller loop body keeps the
@@ -429,7 +494,7 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
     const int r = r0 + rr;
     RowBlock<D, BITS> cur = rbuf[rr];
     if (r + PF < RB) rbuf[rr].load(rec, r + PF, g, t);
-    int d[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
+    int d[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
       uint32_t a[4];
@@ -440,39 +505,39 @@ __device__ __forceinline__ void decode_head(const PoolDev& p, int head, int n, c
         a[2] = ((w0 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
         a[3] = ((w1 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
         mma_u8s8(d, a, bfr[c][0], bfr[c][1]);
-        if constexpr (ADAPT) mma_u8s8(d2, a, bfr2[c][0], bfr2[c][1]);
       } else {
         a[0] = cur.w[0][2 * c];
         a[1] = cur.w[1][2 * c];
         a[2] = cur.w[0][2 * c + 1];
         a[3] = cur.w[1][2 * c + 1];
         mma_s8s8(d, a, bfr[c][0], bfr[c][1]);
-        if constexpr (ADAPT) mma_s8s8(d2, a, bfr2[c][0], bfr2[c][1]);
       }
-    }
-    // digit columns: lane t = 0 holds d0, d1 and lane t = 1 holds d2 of q^
-    // (ADAPT: lanes 2, 3 the same of a^; second product: lanes 0, 1 of b^)
-    const float wB = (t & 1) == 0 ? 256.f : 0.f, wA = (t & 1) == 0 ? 1.f : 65536.f;
-    float pg = wA * (float)(d[0] - cA) + wB * (float)(d[1] - cB);
-    float ph = wA * (float)(d[2] - cA) + wB * (float)(d[3] - cB);
-    pg += __shfl_down_sync(FULL, pg, 1);
-    ph += __shfl_down_sync(FULL, ph, 1);
-    if (t == 0) {
-      scr.y[16 * r + g] = pg * down;
-      scr.y[16 * r + g + 8] = ph * down;
     }
     if constexpr (ADAPT) {
-      if (t == 2) {
+      const float v0 = aw0 * (float)(d[0] - ak0), v1 = aw1 * (float)(d[1] - ak1);
+      const float u0 = aw0 * (float)(d[2] - ak0), u1 = aw1 * (float)(d[3] - ak1);
+      const float pg = (t == 0 ? v0 + v1 : v1) + __shfl_down_sync(FULL, v0, 1);
+      const float ph = (t == 0 ? u0 + u1 : u1) + __shfl_down_sync(FULL, u0, 1);
+      if (t == 0) {
+        scr.y[16 * r + g] = pg * down;
+        scr.y[16 * r + g + 8] = ph * down;
+      } else if (t == 1) {
         scr.ya[16 * r + g] = pg * down_a;
         scr.ya[16 * r + g + 8] = ph * down_a;
+      } else if (t == 2) {
+        scr.yb[16 * r + g] = pg * down_b;
+        scr.yb[16 * r + g + 8] = ph * down_b;
       }
-      float pg2 = wA * (float)(d2[0] - cA2) + wB * (float)(d2[1] - cB2);
-      float ph2 = wA * (float)(d2[2] - cA2) + wB * (float)(d2[3] - cB2);
-      pg2 += __shfl_down_sync(FULL, pg2, 1);
-      ph2 += __shfl_down_sync(FULL, ph2, 1);
+    } else {
+      // digit columns: lane t = 0 holds d0, d1 and lane t = 1 holds d2 of q^
+      const float wB = (t & 1) == 0 ? 256.f : 0.f, wA = (t & 1) == 0 ? 1.f : 65536.f;
+      float pg = wA * (float)(d[0] - cA) + wB * (float)(d[1] - cB);
+      float ph = wA * (float)(d[2] - cA) + wB * (float)(d[3] - cB);
+      pg += __shfl_down_sync(FULL, pg, 1);
+      ph += __shfl_down_sync(FULL, ph, 1);
       if (t == 0) {
-        scr.yb[16 * r + g] = pg2 * down_b;
-        scr.yb[16 * r + g + 8] = ph2 * down_b;
+        scr.y[16 * r + g] = pg * down;
+        scr.y[16 * r + g + 8] = ph * down;
       }
     }
   }
@@ -662,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       reinterpret_cast<WarpScratch<D, ADAPT>*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES)[wib];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarpsPerBlock * NS * ST::BYTES +
                                               kWarpsPerBlock * sizeof(WarpScratch<D, ADAPT>)) + NS * wib;
-  for (int i = lane; i < D; i += 32) scr.dig[3][i] = 0;
+  for (int i = lane; i < D; i += 32) scr.dig[WarpScratch<D, ADAPT>::NDIG - 1][i] = 0;
   const int n_heads = sp.nb * p.H;   // work items of this launch
   const int warp0 = blockIdx.x * kWarpsPerBlock + wib;
   const int W = gridDim.x * kWarpsPerBlock;
