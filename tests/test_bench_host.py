@@ -48,3 +48,15 @@ def test_profiles_hold_traffic_for_the_current_kernel_sources():
         digest = bench.kernel_source_digest(kernel)
         traffic = bench.ncu_traffic(kernel, digest)
         assert traffic is not None and traffic > 0, (kernel, digest)
+
+
+def test_source_digest_ignores_comments_only():
+    """A traffic record stays valid across comment edits and not across code
+    edits: the digest is taken over the code with comments left out."""
+    bench = _bench_module()
+    code = 'int f(int x) {\n  // a comment\n  return x + 1; /* and\n another */\n}\n'
+    same = 'int f(int x) {\n  // another comment entirely\n  return x + 1;\n}\n'
+    changed = 'int f(int x) {\n  return x + 2;\n}\n'
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(changed)
+    assert "comment" not in bench._code_only(code)
