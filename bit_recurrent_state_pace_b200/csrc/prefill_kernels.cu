@@ -89,6 +89,28 @@ __device__ __forceinline__ void stage_chunk(SM& sm, int buf, int64_t c0, int n, 
   cp_async_commit();
 }
 
+// Four 8 x 8 b16 matrices from shared memory (lane l gives the address of
+// row l % 8 of matrix l / 8), as the A fragment of m16n8k16.
+__device__ __forceinline__ void ldsm_x4(const void* row, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(row)));
+}
+// Two 8 x 8 b16 matrices (lanes 0..15 give the row addresses), as the B
+// fragment of m16n8k16 when the rows are B's columns.
+__device__ __forceinline__ void ldsm_x2(const void* row, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"((uint32_t)__cvta_generic_to_shared(row)));
+}
+__device__ __forceinline__ void mma16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Lane L ends with the warp-wide sum of value index (L mod V).
 template <int V>
 __device__ __forceinline__ float transpose_sum(float (&v)[V], int lane) {
@@ -190,7 +212,30 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       b_nx = load_io(beta, row, io);
     }
 
-    // b. dot products in groups of 16 (G: 0..63, M: 64..127), groups strided over warps
+    // b. dot products k_t.k_s (G) and q_t.k_s (M).  bf16 rows: one warp on the
+    //    tensor cores (exact products, fp32 sums), A = [k rows; q rows], B =
+    //    the k rows as columns, while the other warps go on to the operand
+    //    tables.  fp32 rows: lane-parallel sums in groups of 16 (G: 0..63,
+    //    M: 64..127), groups strided over the warps.
+    if constexpr (BF16) {
+      if (w == 0) {
+        float dg[4] = {0.f, 0.f, 0.f, 0.f};
+        const int mq = lane >> 3, rr = lane & 7;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          uint32_t a[4], b0, b1;
+          // matrices: (k rows, cols 16ks..), (q rows, 16ks..), (k rows, 16ks+8..), (q rows, 16ks+8..)
+          ldsm_x4(&sm.raw[buf][mq & 1][rr][2 * (16 * ks + 8 * (mq >> 1))], a);
+          ldsm_x2(&sm.raw[buf][0][rr][2 * (16 * ks + 8 * (mq & 1))], b0, b1);
+          mma16816_bf16(dg, a, b0, b1);
+        }
+        sm.G[g][2 * t] = dg[0];
+        sm.G[g][2 * t + 1] = dg[1];
+        sm.M[g][2 * t] = dg[2];
+        sm.M[g][2 * t + 1] = dg[3];
+        __syncwarp();
+      }
+    } else {
     for (int base = 16 * w; base < 2 * CH * CH; base += 16 * C::RB) {
       float part[16];
 #pragma unroll
@@ -211,6 +256,7 @@ __device__ void prefill_head(const PoolDev& p, int head, int64_t T, const void* 
       }
     }
     __syncthreads();   // dot products ready
+    }
     // warps 1.. build the operand tables while warp 0 forms the chunk scalars
     const int tbl_tid = tid - 32, tbl_n = C::THREADS - 32;
     // K / Q B-fragment tables: entry (x, ks, g, t) of tile x (K, Q, K_lo, Q_lo)
