@@ -186,7 +186,10 @@ pace_status pace_init_pool(const pace_pool_desc* desc, void* d_state, void* d_bu
     dv.bits[h] = desc->head_bits[h];
     p->rec_bytes[h] = L.rec_bytes[h];
   }
-  if (desc->d_k == 128 && desc->d_v == 128)
+  // the tensor stores address a record by its first 64-byte row as a signed
+  // 32-bit coordinate: a state region beyond 2^31 such rows (128 GiB) takes
+  // the mma.sync commit
+  if (desc->d_k == 128 && desc->d_v == 128 && L.state_bytes / 64 <= 0x7fffffffull)
     p->maps_ok = pace::make_commit_maps(dv.state, L.state_bytes, &p->maps);
   // the tensor-memory commit where it is built for the shape, else mma.sync
   p->commit_engine = p->maps_ok && pace::commit_tc_supported(dv) ? PACE_COMMIT_TCGEN05 : PACE_COMMIT_MMA;

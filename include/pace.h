@@ -208,8 +208,8 @@ pace_status pace_commit_period(pace_pool* pool, void* stream);
  *    update and the encode in registers; every pool shape.
  *  PACE_COMMIT_TCGEN05: fifth-generation tensor cores with the update in
  *    tensor memory and the records written back by TMA stores; pools with
- *    d_k = d_v = 128 and column scales (fp32 io only with P <= 8), else
- *    PACE_ERR_UNSUPPORTED.
+ *    d_k = d_v = 128 and column scales (fp32 io only with P <= 8) whose
+ *    state region is at most 128 GiB, else PACE_ERR_UNSUPPORTED.
  * A new pool starts with PACE_COMMIT_TCGEN05 where that engine is built for
  * its shape, else PACE_COMMIT_MMA.
  * Host-only; applies to launches enqueued after the call.  Any other value
