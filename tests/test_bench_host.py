@@ -60,3 +60,32 @@ def test_source_digest_ignores_comments_only():
     assert bench._code_only(code) == bench._code_only(same)
     assert bench._code_only(code) != bench._code_only(changed)
     assert "comment" not in bench._code_only(code)
+
+
+def test_algorithmic_bytes_count_the_pool_as_laid_out():
+    """The roofline's algorithmic bytes against the library's own layout: the
+    records one decode launch reads (and one commit reads and writes once)
+    add up to the pool's state region, and a period's buffered rows (k, v,
+    alpha, beta in the io dtype) to the buffer's row and gate blocks."""
+    sys.path.insert(0, ROOT)
+    import bit_recurrent_state_pace_b200 as pace
+    import pace_synth
+    bench = _bench_module()
+    for name, over in (("concurrency_stress", {}), ("mixed_4_8", {}), ("gdn_layer_4b", {"io_dtype": "f32"})):
+        w = pace_synth.workload(name, **over)
+        bits = pace_synth.head_bits(w, 0)
+        BH = w.B * w.H
+        axis = pace.PACE_SCALE_COL if w.axis == "col" else pace.PACE_SCALE_ROW
+        io = pace.PACE_IO_BF16 if w.io_dtype == "bf16" else pace.PACE_IO_F32
+        state, _, _ = pace.pace_pool_bytes(w.B, w.H, w.d_k, w.d_v, w.P, axis, io, bits)
+        dec1, com, *_ = bench.alg_bytes(w, bits, 1)
+        esz = 2 if w.io_dtype == "bf16" else 4
+        # a decode at buffer position 1: the records, the token in, its row
+        # buffered, o out, the fill read and written
+        per_head = (2 * w.d_k + w.d_v + 2) * esz + (w.d_k + w.d_v + 2) * esz + 4 * w.d_v + 8
+        assert dec1 - BH * per_head == state, name
+        # the commit: every record read and written, P buffered rows read
+        _, buf1, _ = pace.pace_pool_bytes(w.B, w.H, w.d_k, w.d_v, w.P, axis, io, bits)
+        rows = com - 2 * state - 8 * BH
+        assert rows == BH * w.P * (w.d_k + w.d_v + 2) * esz, name
+        assert rows <= buf1, name
